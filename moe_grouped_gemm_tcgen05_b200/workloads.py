@@ -1,0 +1,183 @@
+"""Seeded synthetic inputs shaped like DeepSeek-style dense and MoE layers.
+
+This module only draws random numbers and quantises them to the operand format
+(E4M3 bytes with one power-of-two fp32 scale per block). It holds none of the
+library's arithmetic: it does not pack scales, decode E4M3 or multiply, and it
+never calls the CUDA library. Tests and the benchmark feed the same arrays to
+the CUDA path and to the CPU oracle.
+
+Quantisation recipe (input preparation only): for every block (1x128 along K
+for activations, 128x128 for weights) the scale is
+s = 2^ceil(log2(max(amax, 1e-4) / 448)) and the stored byte is
+``float8_e4m3fn(x / s)`` (round to nearest even, |x / s| <= 448 so nothing
+saturates). Scales are returned as fp32 powers of two, i.e. valid UE8M0
+inputs to the pack step.
+
+Workloads (seed = 1000 + workload number, numpy PCG64):
+  0  dense M=128, N=256, K=512
+  1  dense M in {64, 4096} x (N, K) in {(2112,7168), (24576,1536), (7168,16384), (4096,7168)}
+  2  contiguous, 8 experts, rows per expert U{3072..5120} padded to 128, N=4096, K=7168
+  3  masked, 32 groups, max_m=256, masked_m U{67..124}; up (4096,7168), down (7168,2048)
+  4  masked, 256 groups, max_m=512, masked_m ~ Zipf(1.1) on {0..512}, (7168,2048)
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+BLOCK = 128
+E4M3_MAX = 448.0
+AMAX_FLOOR = 1e-4
+NAN_BYTE = 0x7F  # an E4M3 NaN pattern, used to fill rows that must not be read
+
+DENSE_NK = [(2112, 7168), (24576, 1536), (7168, 16384), (4096, 7168)]
+DENSE_M = [64, 4096]
+
+
+def rng_for(seed: int) -> np.random.Generator:
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _pow2_ceil_ratio(amax: np.ndarray) -> np.ndarray:
+    """2^ceil(log2(max(amax, floor) / 448)) computed exactly with frexp."""
+    v = np.maximum(amax.astype(np.float64), AMAX_FLOOR) / E4M3_MAX
+    mant, exp = np.frexp(v)  # v = mant * 2^exp, mant in [0.5, 1)
+    e = np.where(mant == 0.5, exp - 1, exp)
+    return np.ldexp(1.0, e).astype(np.float32)
+
+
+def _to_e4m3_bytes(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def quantise_rows(x: np.ndarray):
+    """x float32 [R, K] -> (bytes uint8 [R, K], scales float32 [R, K/128])."""
+    R, K = x.shape
+    assert K % BLOCK == 0
+    xb = x.reshape(R, K // BLOCK, BLOCK)
+    s = _pow2_ceil_ratio(np.abs(xb).max(axis=2))
+    q = _to_e4m3_bytes(xb / s[:, :, None]).reshape(R, K)
+    return q, s
+
+
+def quantise_blocks(w: np.ndarray):
+    """w float32 [N, K] -> (bytes uint8 [N, K], scales float32 [ceil(N/128), K/128])."""
+    N, K = w.shape
+    assert K % BLOCK == 0
+    NB = (N + BLOCK - 1) // BLOCK
+    pad = np.zeros((NB * BLOCK, K), dtype=np.float32)
+    pad[:N] = w
+    wb = pad.reshape(NB, BLOCK, K // BLOCK, BLOCK)
+    s = _pow2_ceil_ratio(np.abs(wb).max(axis=(1, 3)))
+    q = _to_e4m3_bytes(wb / s[:, None, :, None]).reshape(NB * BLOCK, K)[:N]
+    return np.ascontiguousarray(q), s
+
+
+def _normal(rng, shape):
+    return rng.standard_normal(size=shape, dtype=np.float32)
+
+
+def dense(M: int, N: int, K: int, seed: int):
+    """Dense NT problem: a [M,K], sfa_f32 [M,K/128], b [N,K], sfb_f32 [ceil(N/128),K/128]."""
+    rng = rng_for(seed)
+    a, sfa = quantise_rows(_normal(rng, (M, K)))
+    b, sfb = quantise_blocks(_normal(rng, (N, K)))
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, M=M, N=N, K=K)
+
+
+def grouped_weights(rng, G: int, N: int, K: int):
+    bs, sfbs = [], []
+    for _ in range(G):
+        b, sfb = quantise_blocks(_normal(rng, (N, K)))
+        bs.append(b)
+        sfbs.append(sfb)
+    return np.stack(bs), np.stack(sfbs)
+
+
+def contiguous(counts, N: int, K: int, seed: int, align: int = BLOCK, tail_blocks: int = 0):
+    """Contiguous M-grouped problem.
+
+    Expert g owns ``counts[g]`` real rows, padded with -1 rows up to a multiple
+    of ``align``; ``tail_blocks`` extra all-padding blocks are appended. Padding
+    rows of A hold NaN bytes.
+    """
+    rng = rng_for(seed)
+    G = len(counts)
+    seg = [((c + align - 1) // align) * align for c in counts]
+    M_total = int(sum(seg)) + tail_blocks * align
+    m_indices = np.full(M_total, -1, dtype=np.int32)
+    off = 0
+    for g, (c, s) in enumerate(zip(counts, seg)):
+        m_indices[off:off + c] = g
+        off += s
+    a = np.full((M_total, K), NAN_BYTE, dtype=np.uint8)
+    sfa = np.ones((M_total, K // BLOCK), dtype=np.float32)
+    valid = m_indices >= 0
+    qa, qs = quantise_rows(_normal(rng, (int(valid.sum()), K)))
+    a[valid] = qa
+    sfa[valid] = qs
+    b, sfb = grouped_weights(rng, G, N, K)
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, m_indices=m_indices,
+                M_total=M_total, N=N, K=K, G=G)
+
+
+def masked(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bool = True):
+    """Masked M-grouped problem: a [G,max_m,K], b [G,N,K]; rows >= masked_m hold NaN bytes."""
+    rng = rng_for(seed)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = masked_m.shape[0]
+    x = _normal(rng, (G * max_m, K))
+    a, sfa = quantise_rows(x)
+    a = a.reshape(G, max_m, K)
+    sfa = sfa.reshape(G, max_m, K // BLOCK)
+    if fill_invalid_nan:
+        rows = np.arange(max_m)[None, :] >= np.clip(masked_m, 0, max_m)[:, None]
+        a[rows] = NAN_BYTE
+    b, sfb = grouped_weights(rng, G, N, K)
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, masked_m=masked_m,
+                G=G, max_m=max_m, N=N, K=K)
+
+
+# ---- the five workloads -------------------------------------------------
+
+def workload0():
+    return dense(128, 256, 512, seed=1000)
+
+
+def workload1(M: int, N: int, K: int):
+    return dense(M, N, K, seed=1001)
+
+
+def contiguous_counts(seed: int = 1002, G: int = 8, lo: int = 3072, hi: int = 5120):
+    return rng_for(seed).integers(lo, hi + 1, size=G)
+
+
+def workload2():
+    counts = contiguous_counts()
+    return contiguous(counts, 4096, 7168, seed=1002)
+
+
+def masked_m_uniform(rng, G: int = 32, expected: int = 96):
+    lo, hi = int(np.floor(0.7 * expected)), int(np.floor(1.3 * expected))
+    return rng.integers(lo, hi + 1, size=G).astype(np.int32)
+
+
+def workload3(proj: str):
+    N, K = (4096, 7168) if proj == "up" else (7168, 2048)
+    mm = masked_m_uniform(rng_for(1003))
+    return masked(mm, 256, N, K, seed=1003)
+
+
+def zipf_masked_m(rng, G: int = 256, max_m: int = 512, a: float = 1.1):
+    """masked_m drawn with p(m) proportional to (m+1)^-a on {0..max_m}."""
+    m = np.arange(max_m + 1)
+    p = (m + 1.0) ** (-a)
+    p /= p.sum()
+    return rng.choice(m, size=G, p=p).astype(np.int32)
+
+
+def workload4():
+    mm = zipf_masked_m(rng_for(1004))
+    return masked(mm, 512, 7168, 2048, seed=1004, fill_invalid_nan=False)

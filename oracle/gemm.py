@@ -1,0 +1,163 @@
+"""Dequantise-and-multiply references for the three GEMM forms (oracle; test infrastructure only).
+
+What is computed
+----------------
+All three forms compute D = A . B^T with A row-major [rows, K] and B row-major
+[N, K] ("NT"): "DeepInside DeepGEMM", §4 Hands-on Geek Guide, where the
+standard non-grouped FP8 NT GEMM computes D = C + A @ B.T (C is absent here,
+i.e. zero) and returns bf16.
+
+Operands are E4M3 bytes with power-of-two scales stored as packed UE8M0
+(§2 of the same page): activations carry one scale per 1x128 block along K,
+weights one per 128x128 block. The dequantised operands are
+
+    A^[m, k] = e4m3(a[m, k]) * 2^(ea[m, k // 128] - 127)
+    B^[n, k] = e4m3(b[n, k]) * 2^(eb[n // 128, k // 128] - 127)
+
+where ea / eb are the bytes of the packed int32 scale rows (byte j of word i is
+K-block 4*i + j). The reference result is A^ . B^^T in float64.
+
+Grouped forms (readings; the pages name them but print no definition beyond
+the call shape):
+* contiguous: rows of A are concatenated by expert; ``m_indices[r]`` gives the
+  expert of row r. Rows with an index outside [0, G) (-1 marks padding) are
+  not computed and their output is left as it was.
+* masked ("DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs",
+  Tensor-Based Metadata Arguments and the FAQ on dynamic shapes): A is
+  [G, max_m, K] and D is [G, max_m, N]; only the first masked_m[g] rows of group
+  g are valid (masked_m clamped to [0, max_m]); every other row of D is left as
+  it was.
+
+Each grouped reference returns (values, valid) where ``valid`` marks the rows
+whose output is defined; rows outside it must keep their previous bits.
+"""
+
+import numpy as np
+
+from .fp8 import e4m3_to_f64
+from .ue8m0 import ue8m0_to_f64, unpack_ue8m0
+
+BLOCK = 128  # scale granularity along K (and along N for the weights)
+
+
+def _kb(K: int) -> int:
+    if K % BLOCK != 0:
+        raise ValueError(f"K={K} is not a multiple of {BLOCK}")
+    return K // BLOCK
+
+
+def dequant_rows(a, sfa) -> np.ndarray:
+    """A^ for activation rows: a uint8 [R, K], sfa int32 [R, KP] -> float64 [R, K]."""
+    a = np.asarray(a, dtype=np.uint8)
+    R, K = a.shape
+    KB = _kb(K)
+    scale = ue8m0_to_f64(unpack_ue8m0(sfa, KB))  # [R, KB], one per 1x128 block
+    vals = e4m3_to_f64(a).reshape(R, KB, BLOCK)
+    return (vals * scale[:, :, None]).reshape(R, K)
+
+
+def dequant_weights(b, sfb, cols=None) -> np.ndarray:
+    """B^ for weight rows: b uint8 [N, K], sfb int32 [ceil(N/128), KP] -> float64.
+
+    ``cols`` (optional) selects which rows n of B to dequantise, so that sampled
+    checks need not expand the whole weight.
+    """
+    b = np.asarray(b, dtype=np.uint8)
+    N, K = b.shape
+    KB = _kb(K)
+    n = np.arange(N) if cols is None else np.asarray(cols, dtype=np.int64)
+    block_scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))  # [ceil(N/128), KB]
+    scale = block_scale[n // BLOCK]  # one per 128x128 block
+    vals = e4m3_to_f64(b[n]).reshape(len(n), KB, BLOCK)
+    return (vals * scale[:, :, None]).reshape(len(n), K)
+
+
+def fp8_gemm_nt(a, sfa, b, sfb) -> np.ndarray:
+    """Dense D[M, N] = A^ . B^^T in float64."""
+    return dequant_rows(a, sfa) @ dequant_weights(b, sfb).T
+
+
+def fp8_gemm_nt_sampled(a, sfa, b, sfb, rows, cols) -> np.ndarray:
+    """D[rows[i], cols[i]] of the dense GEMM, one output at a time (float64)."""
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    ur, ri = np.unique(rows, return_inverse=True)
+    uc, ci = np.unique(cols, return_inverse=True)
+    ah = dequant_rows(np.asarray(a)[ur], np.asarray(sfa)[ur])
+    bh = dequant_weights(b, sfb, cols=uc)
+    return np.einsum("ik,ik->i", ah[ri], bh[ci])
+
+
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices):
+    """Contiguous M-grouped GEMM.
+
+    a uint8 [M_total, K], sfa int32 [M_total, KP], b uint8 [G, N, K],
+    sfb int32 [G, ceil(N/128), KP], m_indices int32 [M_total].
+    Returns (D float64 [M_total, N] with NaN on undefined rows, valid bool [M_total]).
+    """
+    b = np.asarray(b, dtype=np.uint8)
+    G, N, _ = b.shape
+    m_indices = np.asarray(m_indices, dtype=np.int64)
+    M_total = m_indices.shape[0]
+    out = np.full((M_total, N), np.nan, dtype=np.float64)
+    valid = (m_indices >= 0) & (m_indices < G)
+    for g in range(G):
+        r = np.nonzero(m_indices == g)[0]
+        if r.size == 0:
+            continue
+        out[r] = dequant_rows(np.asarray(a)[r], np.asarray(sfa)[r]) @ dequant_weights(b[g], np.asarray(sfb)[g]).T
+    return out, valid
+
+
+def m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, cols):
+    """Sampled outputs of the contiguous GEMM; rows must have a valid expert."""
+    m_indices = np.asarray(m_indices, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    out = np.empty(rows.shape[0], dtype=np.float64)
+    g_of = m_indices[rows]
+    if np.any((g_of < 0) | (g_of >= np.asarray(b).shape[0])):
+        raise ValueError("sampled rows must belong to an expert")
+    for g in np.unique(g_of):
+        sel = np.nonzero(g_of == g)[0]
+        out[sel] = fp8_gemm_nt_sampled(a, sfa, np.asarray(b)[g], np.asarray(sfb)[g], rows[sel], cols[sel])
+    return out
+
+
+def masked_valid_rows(masked_m, G: int, max_m: int) -> np.ndarray:
+    """valid[g, r] = r < clamp(masked_m[g], 0, max_m)."""
+    mm = np.clip(np.asarray(masked_m, dtype=np.int64), 0, max_m)
+    return np.arange(max_m)[None, :] < mm[:G, None]
+
+
+def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m):
+    """Masked M-grouped GEMM.
+
+    a uint8 [G, max_m, K], sfa int32 [G, max_m, KP], b uint8 [G, N, K],
+    sfb int32 [G, ceil(N/128), KP], masked_m int32 [G].
+    Returns (D float64 [G, max_m, N] with NaN on undefined rows, valid bool [G, max_m]).
+    """
+    a = np.asarray(a, dtype=np.uint8)
+    G, max_m, _ = a.shape
+    N = np.asarray(b).shape[1]
+    valid = masked_valid_rows(masked_m, G, max_m)
+    out = np.full((G, max_m, N), np.nan, dtype=np.float64)
+    for g in range(G):
+        m = int(valid[g].sum())
+        if m == 0:
+            continue
+        out[g, :m] = fp8_gemm_nt(a[g, :m], np.asarray(sfa)[g, :m], np.asarray(b)[g], np.asarray(sfb)[g])
+    return out, valid
+
+
+def m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, groups, rows, cols):
+    """Sampled outputs D[groups[i], rows[i], cols[i]] of the masked GEMM (valid rows only)."""
+    groups = np.asarray(groups, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    out = np.empty(groups.shape[0], dtype=np.float64)
+    for g in np.unique(groups):
+        sel = np.nonzero(groups == g)[0]
+        out[sel] = fp8_gemm_nt_sampled(np.asarray(a)[g], np.asarray(sfa)[g], np.asarray(b)[g],
+                                       np.asarray(sfb)[g], rows[sel], cols[sel])
+    return out

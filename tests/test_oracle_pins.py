@@ -1,0 +1,323 @@
+"""Pins for the CPU oracle, independent of the oracle itself (CPU only).
+
+Each pin checks the oracle against something it does not compute itself:
+worked examples derived by hand from the pack formula in "[GH-ISSUE #414]
+pack_ue8m0_to_int is not CUDA Graph capture safe", the OCP E4M3 definition
+(spot values, and torch's own float8 decode for all 256 codes), closed forms
+(one-hot operands, powers of two), exact rational brute force on tiny shapes,
+and special cases that reduce to a library matmul. The last tests plant
+mistakes in a copy of the oracle and check that the pins catch them.
+"""
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import gemm as og
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def torch_e4m3(codes):
+    """torch's float8_e4m3fn decode of byte codes, as float64 (library routine)."""
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(codes, dtype=np.uint8)))
+    return t.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------- E4M3 ----
+
+def test_e4m3_spot_values_from_ocp_definition():
+    spots = {
+        0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+        0x38: 1.0, 0x3C: 1.5, 0x40: 2.0, 0x7E: 448.0,
+        0x80: -0.0, 0xB8: -1.0, 0xFE: -448.0,
+    }
+    for code, want in spots.items():
+        got = oracle.e4m3_to_f64(np.array([code]))[0]
+        assert got == want and math.copysign(1, got) == math.copysign(1, want), hex(code)
+    assert np.isnan(oracle.e4m3_to_f64(np.array([0x7F, 0xFF]))).all()
+    assert oracle.E4M3_MAX == 448.0
+
+
+def test_e4m3_table_matches_torch_float8_decode():
+    codes = np.arange(256)
+    mine = oracle.e4m3_to_f64(codes)
+    ref = torch_e4m3(codes)
+    same = (mine == ref) | (np.isnan(mine) & np.isnan(ref))
+    assert same.all(), codes[~same]
+
+
+# --------------------------------------------------------------- UE8M0 ----
+
+def test_ue8m0_decode_closed_form():
+    v = oracle.ue8m0_to_f64(np.array([0, 1, 126, 127, 128, 254, 255]))
+    assert v[0] == 2.0 ** -127 and v[1] == 2.0 ** -126
+    assert v[2] == 0.5 and v[3] == 1.0 and v[4] == 2.0 and v[5] == 2.0 ** 127
+    assert np.isnan(v[6])
+
+
+def _read_pack_golden():
+    cases = []
+    with open(os.path.join(GOLDEN, "pack_ue8m0_worked.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            scales, byts, word = [p.strip() for p in line.split("|")]
+            cases.append(([float(s) for s in scales.split()],
+                          [int(x, 16) for x in byts.split()], int(word, 16)))
+    return cases
+
+
+def test_pack_matches_hand_worked_examples():
+    cases = _read_pack_golden()
+    assert len(cases) >= 4
+    for scales, byts, word in cases:
+        got = oracle.pack_ue8m0(np.array([scales], dtype=np.float32))
+        assert got.shape == (1, 1)
+        assert (int(got[0, 0]) & 0xFFFFFFFF) == word, (scales, hex(int(got[0, 0]) & 0xFFFFFFFF))
+        assert list(oracle.unpack_ue8m0(got, 4)[0]) == byts
+
+
+def test_pack_every_finite_positive_power_of_two():
+    # all 254 normal powers of two 2^-126 .. 2^127: byte = e + 127, and it decodes back exactly
+    e = np.arange(-126, 128)
+    sf = np.ldexp(np.float32(1.0), e).astype(np.float32)
+    n = sf.size
+    cols = 4 * ((n + 3) // 4)
+    grid = np.ones(cols, dtype=np.float32)
+    grid[:n] = sf
+    packed = oracle.pack_ue8m0(grid.reshape(1, cols))
+    byts = oracle.unpack_ue8m0(packed, cols)[0, :n]
+    assert (byts.astype(np.int64) == e + 127).all()
+    assert (oracle.ue8m0_to_f64(byts) == sf.astype(np.float64)).all()
+    assert oracle.pack_ue8m0_validate(grid.reshape(1, cols)) == 0
+
+
+def test_pack_ragged_columns_pad_with_zero_bytes():
+    sf = np.array([[2.0, 4.0, 8.0, 16.0, 0.5, 0.25]], dtype=np.float32)
+    p = oracle.pack_ue8m0(sf)
+    assert p.shape == (1, 2)
+    assert (int(p[0, 1]) & 0xFFFFFFFF) == 0x00007D7E  # bytes 7E 7D 00 00
+    assert (int(p[0, 0]) & 0xFFFFFFFF) == 0x83828180
+
+
+def test_validator_counts_issue_conditions():
+    sf = np.array([[1.0, -1.0, 3.0, 0.0, float("inf"), 1.5, -0.0, 2.0 ** -20]], dtype=np.float32)
+    # sign set: -1.0, -0.0 ; mantissa != 0: 3.0, 1.5
+    assert oracle.pack_ue8m0_validate(sf) == 4
+
+
+# ---------------------------------------------------------------- GEMM ----
+
+def _rand_codes(rng, shape, lo_exp=4, hi_exp=11):
+    """E4M3 codes with exponent field in [lo_exp, hi_exp] and random sign/mantissa."""
+    s = rng.integers(0, 2, size=shape)
+    e = rng.integers(lo_exp, hi_exp + 1, size=shape)
+    m = rng.integers(0, 8, size=shape)
+    return ((s << 7) | (e << 3) | m).astype(np.uint8)
+
+
+def _pack_bytes(byts):
+    """Pack a uint8 [rows, cols] array of UE8M0 bytes into int32 words (test-side, little-endian)."""
+    rows, cols = byts.shape
+    kp = (cols + 3) // 4
+    w = np.zeros((rows, kp), dtype=np.int64)
+    for c in range(cols):
+        w[:, c // 4] |= byts[:, c].astype(np.int64) << (8 * (c % 4))
+    return w.astype(np.uint32).view(np.int32)
+
+
+def _exact_gemm(a, ea, b, eb):
+    """Exact rational D = A^ B^^T with explicit block loops (no shared code with the oracle)."""
+    M, K = a.shape
+    N = b.shape[0]
+    av = torch_e4m3(a)
+    bv = torch_e4m3(b)
+    out = [[Fraction(0)] * N for _ in range(M)]
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for kb in range(K // 128):
+                sa = Fraction(2) ** (int(ea[m, kb]) - 127)
+                sb = Fraction(2) ** (int(eb[n // 128, kb]) - 127)
+                part = Fraction(0)
+                for kk in range(128):
+                    k = kb * 128 + kk
+                    part += Fraction(av[m, k]) * Fraction(bv[n, k])
+                acc += part * sa * sb
+            out[m][n] = acc
+    return out
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(3, 5, 128, 1), (8, 7, 256, 2), (1, 8, 256, 3)])
+def test_dense_equals_exact_rational_brute_force(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    ea = rng.integers(124, 131, size=(M, K // 128)).astype(np.uint8)
+    eb = rng.integers(124, 131, size=((N + 127) // 128, K // 128)).astype(np.uint8)
+    got = oracle.fp8_gemm_nt(a, _pack_bytes(ea), b, _pack_bytes(eb))
+    exact = _exact_gemm(a, ea, b, eb)
+    for m in range(M):
+        for n in range(N):
+            assert Fraction(got[m, n]) == exact[m][n], (m, n)
+
+
+def test_dense_multi_block_n_exact():
+    # N spans two 128-row weight blocks with different scales; checks the n // 128 index
+    rng = np.random.default_rng(7)
+    M, N, K = 2, 130, 256
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    ea = rng.integers(125, 130, size=(M, 2)).astype(np.uint8)
+    eb = np.array([[126, 129], [131, 123]], dtype=np.uint8)
+    got = oracle.fp8_gemm_nt(a, _pack_bytes(ea), b, _pack_bytes(eb))
+    exact = _exact_gemm(a, ea, b, eb)
+    for m in range(M):
+        for n in (0, 1, 126, 127, 128, 129):
+            assert Fraction(got[m, n]) == exact[m][n], (m, n)
+
+
+def one_hot_check(gemm_fn) -> bool:
+    """D of one-hot A rows must be exactly 2^pa * b[n, k_m] * 2^pb(n // 128, k_m // 128)."""
+    rng = np.random.default_rng(11)
+    M, N, K = 6, 300, 640  # 5 K-blocks (ragged packing), 3 N-blocks
+    KB, NB = K // 128, 3
+    ks = np.array([0, 127, 128, 300, 511, 639])
+    a = np.zeros((M, K), dtype=np.uint8)
+    a[np.arange(M), ks] = 0x38  # 1.0
+    ea = np.full((M, KB), 127, dtype=np.uint8)
+    pa = np.array([0, 3, -2, 5, 1, -4])
+    ea[np.arange(M), ks // 128] = 127 + pa
+    b = _rand_codes(rng, (N, K))
+    eb = rng.integers(120, 135, size=(NB, KB)).astype(np.uint8)
+    got = gemm_fn(a, _pack_bytes(ea), b, _pack_bytes(eb))
+    bv = torch_e4m3(b)
+    n = np.arange(N)
+    for m in range(M):
+        want = (2.0 ** pa[m]) * bv[n, ks[m]] * np.ldexp(1.0, eb[n // 128, ks[m] // 128].astype(np.int64) - 127)
+        if got.shape != (M, N) or not np.array_equal(got[m], want):
+            return False
+    return True
+
+
+def test_one_hot_rows_exact():
+    assert one_hot_check(oracle.fp8_gemm_nt)
+
+
+def test_identity_times_b_is_b_scaled():
+    # A = I (128x128, one 1x128 block per row), unit A scales -> D = B^ exactly
+    rng = np.random.default_rng(5)
+    N, K = 200, 128
+    a = np.where(np.eye(K, dtype=bool), 0x38, 0x00).astype(np.uint8)
+    b = _rand_codes(rng, (N, K))
+    eb = np.array([[129], [125]], dtype=np.uint8)
+    d = oracle.fp8_gemm_nt(a, _pack_bytes(np.full((K, 1), 127, np.uint8)), b, _pack_bytes(eb))
+    want = (torch_e4m3(b) * np.ldexp(1.0, eb[np.arange(N) // 128, 0].astype(np.int64) - 127)[:, None]).T
+    assert np.array_equal(d, want)
+
+
+def test_unit_scales_reduce_to_plain_matmul():
+    rng = np.random.default_rng(9)
+    M, N, K = 37, 150, 384
+    a = _rand_codes(rng, (M, K), 0, 14)
+    b = _rand_codes(rng, (N, K), 0, 14)
+    ones_a = _pack_bytes(np.full((M, 3), 127, np.uint8))
+    ones_b = _pack_bytes(np.full((2, 3), 127, np.uint8))
+    got = oracle.fp8_gemm_nt(a, ones_a, b, ones_b)
+    ref = (torch.from_numpy(torch_e4m3(a)) @ torch.from_numpy(torch_e4m3(b)).T).numpy()
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-9)
+
+
+def test_sampled_matches_full():
+    rng = np.random.default_rng(3)
+    M, N, K = 20, 260, 512
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(rng.integers(120, 135, size=(M, 4)).astype(np.uint8))
+    sfb = _pack_bytes(rng.integers(120, 135, size=(3, 4)).astype(np.uint8))
+    full = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    r = rng.integers(0, M, size=50)
+    c = rng.integers(0, N, size=50)
+    assert np.array_equal(oracle.fp8_gemm_nt_sampled(a, sfa, b, sfb, r, c), full[r, c])
+
+
+def test_masked_rows_and_clamp():
+    rng = np.random.default_rng(4)
+    G, max_m, N, K = 4, 9, 130, 256
+    a = _rand_codes(rng, (G, max_m, K))
+    b = _rand_codes(rng, (G, N, K))
+    sfa = _pack_bytes(rng.integers(120, 135, size=(G * max_m, 2)).astype(np.uint8)).reshape(G, max_m, 1)
+    sfb = _pack_bytes(rng.integers(120, 135, size=(G * 2, 2)).astype(np.uint8)).reshape(G, 2, 1)
+    masked_m = np.array([3, -5, 100, 0], dtype=np.int32)
+    d, valid = oracle.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m)
+    assert valid.sum(axis=1).tolist() == [3, 0, max_m, 0]
+    assert np.isnan(d[~valid]).all()
+    for g in range(G):
+        m = int(valid[g].sum())
+        if m:
+            assert np.array_equal(d[g, :m], oracle.fp8_gemm_nt(a[g, :m], sfa[g, :m], b[g], sfb[g]))
+    # a single full group is exactly the dense GEMM
+    d1, _ = oracle.m_grouped_fp8_gemm_nt_masked(a[2:3], sfa[2:3], b[2:3], sfb[2:3], np.array([max_m]))
+    assert np.array_equal(d1[0], oracle.fp8_gemm_nt(a[2], sfa[2], b[2], sfb[2]))
+
+
+def test_contiguous_rows_follow_their_expert():
+    rng = np.random.default_rng(6)
+    G, N, K = 3, 140, 256
+    m_indices = np.array([0] * 5 + [-1] * 3 + [2] * 4 + [1] * 2 + [-1] * 2, dtype=np.int32)
+    Mt = m_indices.size
+    a = _rand_codes(rng, (Mt, K))
+    b = _rand_codes(rng, (G, N, K))
+    sfa = _pack_bytes(rng.integers(120, 135, size=(Mt, 2)).astype(np.uint8))
+    sfb = _pack_bytes(rng.integers(120, 135, size=(G * 2, 2)).astype(np.uint8)).reshape(G, 2, 1)
+    d, valid = oracle.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices)
+    assert np.array_equal(valid, m_indices >= 0)
+    assert np.isnan(d[~valid]).all()
+    for r in np.nonzero(valid)[0]:
+        g = m_indices[r]
+        assert np.array_equal(d[r], oracle.fp8_gemm_nt(a[r:r + 1], sfa[r:r + 1], b[g], sfb[g])[0])
+    rows = np.nonzero(valid)[0]
+    cols = rng.integers(0, N, size=rows.size)
+    s = oracle.m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, cols)
+    assert np.array_equal(s, d[rows, cols])
+
+
+# ----------------------------------------------------- planted mistakes ----
+
+def _planted(kind):
+    """A copy of the dense oracle with one plausible mistake planted (CPU only)."""
+    def fn(a, sfa, b, sfb):
+        A = og.dequant_rows(a, sfa)
+        if kind == "weight_scale_per_row":
+            # B scale indexed by n instead of n // 128
+            N, K = b.shape
+            KB = K // 128
+            s = oracle.ue8m0_to_f64(oracle.unpack_ue8m0(sfb, KB))
+            idx = np.minimum(np.arange(N), s.shape[0] - 1)
+            B = (oracle.e4m3_to_f64(b).reshape(N, KB, 128) * s[idx][:, :, None]).reshape(N, K)
+        else:
+            B = og.dequant_weights(b, sfb)
+        if kind == "byte_order_reversed":
+            M, K = A.shape
+            KB = K // 128
+            rev = oracle.unpack_ue8m0(sfa, 4 * sfa.shape[1]).reshape(M, -1, 4)[:, :, ::-1].reshape(M, -1)[:, :KB]
+            A = (oracle.e4m3_to_f64(a).reshape(M, KB, 128) * oracle.ue8m0_to_f64(rev)[:, :, None]).reshape(M, K)
+        if kind == "transposed_b":
+            return A @ B[:, : A.shape[1]].T if B.shape[1] != A.shape[1] else (A @ B.T)[:, ::-1]
+        if kind == "dropped_last_block":
+            A = A.copy()
+            A[:, -128:] = 0
+        return A @ B.T
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["weight_scale_per_row", "byte_order_reversed", "transposed_b", "dropped_last_block"])
+def test_pins_catch_planted_mistakes(kind):
+    assert not one_hot_check(_planted(kind)), kind
