@@ -1,0 +1,183 @@
+/*
+ * dgb200 -- FP8 (E4M3) block-scaled GEMMs and the UE8M0 scale pack for B200 (sm_100a).
+ *
+ * C ABI of libdgb200.so. Every argument is a plain pointer or an integer; no
+ * framework type appears here. Device pointers point to memory on the current
+ * CUDA device; `stream` is a cudaStream_t passed as void* (NULL = legacy
+ * default stream).
+ *
+ * Operation (all three GEMM forms): D = A . B^T ("NT"), E4M3 operands, fp32
+ * accumulation, bf16 output, no C term. Sources: "DeepInside DeepGEMM:
+ * Unpacking DeepSeek's Unified Tensor Core Library for SM90 and SM100",
+ * section 4 (the standard non-grouped FP8 NT GEMM computes D = C + A @ B.T)
+ * and section 2 (on SM100 the scaling factors are UE8M0, four packed into one
+ * torch.int).
+ *
+ * Scales. Activations (A) carry one scale per 1x128 block along K, weights (B)
+ * one scale per 128x128 block. A scale is a UE8M0 byte e meaning 2^(e-127).
+ * Scale rows are packed four bytes per int32, little-endian, consecutive
+ * along K: byte j of word i is K-block 4*i + j. With KB = K/128 and
+ * KP = ceil(KB/4):
+ *     sfa: int32 [rows, KP]            row-major, one row per row of A
+ *     sfb: int32 [ceil(N/128), KP]     row-major, one row per 128 rows of B
+ * pack_ue8m0() produces exactly this layout from fp32 scales.
+ *
+ * Layouts. All tensors are dense and row-major. A rows are K bytes long, B rows
+ * K bytes, D rows N bf16 values.
+ *
+ * Ownership. The caller allocates and owns every buffer. The library keeps no
+ * per-call state and allocates no device memory in any call.
+ *
+ * CUDA Graph capture. Every compute entry point is capture safe: no host
+ * synchronisation, no allocation, no host reads of device values, and a launch
+ * configuration fixed by the scalar sizes alone ("DeepGEMM CUDA Graph
+ * Compatibility for Masked Grouped GEMMs: Implementation Guide", sections
+ * Stateless Kernel Architecture and Tensor-Based Metadata Arguments). All
+ * variable metadata (masked_m, m_indices, scales) is read on the device. The
+ * first call on a device configures the kernels (cudaFuncSetAttribute); make
+ * it, or dgb200_init(), before capturing.
+ *
+ * Errors. Host-checkable mistakes return a status without launching anything:
+ * null pointers, non-positive sizes, K not a multiple of 128, N not a multiple
+ * of 8, misaligned pointers (A, B, D need 16-byte alignment; scales and
+ * metadata 4-byte), sizes past the limits below. A failed launch returns
+ * DG_ERR_CUDA. Device values are never checked on the host; the kernels
+ * clamp them (see each call) and record problems in a device status word that
+ * dgb200_device_error() reads. Every wait inside a kernel is bounded: a wait
+ * that runs out sets DG_DEVERR_TIMEOUT and the kernel returns instead of
+ * hanging.
+ *
+ * Limits: 1 <= M, N; N % 8 == 0; K % 128 == 0; 128 <= K <= 2^20;
+ * rows * K < 2^40 for every operand; G <= 1024 for the masked form.
+ */
+#ifndef DGB200_H
+#define DGB200_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DG_API __attribute__((visibility("default")))
+#else
+#define DG_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DG_OK = 0,
+    DG_ERR_INVALID_ARG = 1,    /* null pointer, bad size or bad combination */
+    DG_ERR_ALIGNMENT = 2,      /* pointer or row pitch not aligned as required */
+    DG_ERR_UNSUPPORTED = 3,    /* valid request outside this build's limits */
+    DG_ERR_NOT_INITIALIZED = 4,/* no usable CUDA device / driver entry point */
+    DG_ERR_CUDA = 5            /* a CUDA runtime call or launch failed */
+} dg_status;
+
+/* Bits of the device status word (see dgb200_device_error). */
+#define DG_DEVERR_TIMEOUT             1u /* a bounded wait inside a kernel ran out */
+#define DG_DEVERR_MIXED_EXPERT_BLOCK  2u /* contiguous: an aligned 128-row block held two experts */
+
+/* Human-readable name of a status code (static string). */
+DG_API const char* dgb200_status_string(dg_status s);
+
+/*
+ * Configure the kernels for the current device: caches the SM count and sets
+ * the dynamic shared-memory limits. Idempotent and thread safe. Called
+ * implicitly by the first compute call on a device; call it eagerly before any
+ * CUDA Graph capture.
+ */
+DG_API dg_status dgb200_init(void);
+
+/*
+ * Read the device status word of the current device into *bits (host pointer)
+ * and, if clear != 0, reset it to zero. Synchronises the device: never call it
+ * inside a stream capture.
+ */
+DG_API dg_status dgb200_device_error(uint32_t* bits, int clear);
+
+/*
+ * Force the N tile width of the GEMM kernels (0 restores the built-in
+ * heuristic). Allowed widths: see dgb200_block_n_supported(). Process-wide;
+ * meant for tests and tuning.
+ */
+DG_API dg_status dgb200_set_block_n(int block_n);
+DG_API int dgb200_block_n_supported(int block_n);
+
+/*
+ * Dense FP8 NT GEMM ("DeepInside DeepGEMM", section 4: fp8_gemm_nt).
+ *   a   : device, E4M3 [M, K]
+ *   sfa : device, int32 [M, KP]             packed UE8M0, one per 1x128 block
+ *   b   : device, E4M3 [N, K]
+ *   sfb : device, int32 [ceil(N/128), KP]   packed UE8M0, one per 128x128 block
+ *   d   : device, bf16 [M, N]               written completely
+ */
+DG_API dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                      void* d, int M, int N, int K, void* stream);
+
+/*
+ * Contiguous M-grouped FP8 GEMM for MoE ("DeepGEMM tested by Novita AI",
+ * grouped GEMM with continuous storage layout, used for training forward and
+ * prefill). Rows of A are concatenated by expert; m_indices[r] is the expert
+ * of row r, -1 on padding rows.
+ *   a         : device, E4M3 [M_total, K]
+ *   sfa       : device, int32 [M_total, KP]
+ *   b         : device, E4M3 [G, N, K]
+ *   sfb       : device, int32 [G, ceil(N/128), KP]
+ *   d         : device, bf16 [M_total, N]
+ *   m_indices : device, int32 [M_total]
+ * Contract: rows form aligned 128-row blocks (rows 128*i .. 128*i+127); within
+ * a block every row whose index lies in [0, G) names the same expert. Rows with
+ * an index outside [0, G) are padding: they are not computed and their rows of
+ * D are left untouched. A block holding two experts computes only the rows of
+ * the larger index, leaves the others untouched and sets
+ * DG_DEVERR_MIXED_EXPERT_BLOCK.
+ */
+DG_API dg_status m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa,
+                                           const void* b, const int32_t* sfb,
+                                           void* d, const int32_t* m_indices,
+                                           int M_total, int N, int K, int G, void* stream);
+
+/*
+ * Masked M-grouped FP8 GEMM for MoE decode ("DeepGEMM CUDA Graph Compatibility
+ * for Masked Grouped GEMMs", Tensor-Based Metadata Arguments: masked_m is a
+ * device tensor and max_m_per_group a host integer).
+ *   a        : device, E4M3 [G, max_m, K]
+ *   sfa      : device, int32 [G, max_m, KP]
+ *   b        : device, E4M3 [G, N, K]
+ *   sfb      : device, int32 [G, ceil(N/128), KP]
+ *   d        : device, bf16 [G, max_m, N]
+ *   masked_m : device, int32 [G]; group g uses its first masked_m[g] rows,
+ *              clamped on the device to [0, max_m].
+ * Rows at or beyond masked_m[g] are never read for output and their rows of D
+ * are never written (a pre-filled sentinel survives). The grid depends only on
+ * (G, max_m, N, K), so a captured graph can be replayed with new masked_m.
+ */
+DG_API dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa,
+                                       const void* b, const int32_t* sfb,
+                                       void* d, const int32_t* masked_m,
+                                       int G, int max_m, int N, int K, void* stream);
+
+/*
+ * Capture-safe UE8M0 pack ("[GH-ISSUE #414] pack_ue8m0_to_int is not CUDA Graph
+ * capture safe", Expected behavior). For fp32 scales sf [rows, cols] writes
+ * packed [rows, ceil(cols/4)] int32 with byte (bits(sf[r][c]) >> 23) & 0xFF at
+ * byte c % 4 of word c / 4 (zero bytes complete the last word). No value
+ * checks: a scale that is not a positive power of two packs to its exponent
+ * field. Both pointers are device pointers, 4-byte aligned.
+ */
+DG_API dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int cols, void* stream);
+
+/*
+ * Optional validation of the same scales, kept off the pack path as the issue
+ * asks: writes to *bad_count (device int32) the number of entries whose sign
+ * bit is set or whose mantissa is non-zero. Capture safe (the result stays on
+ * the device).
+ */
+DG_API dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* bad_count, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DGB200_H */

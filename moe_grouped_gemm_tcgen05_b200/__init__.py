@@ -1,0 +1,223 @@
+"""FP8 block-scaled GEMMs (dense, contiguous and masked M-grouped) and the UE8M0
+pack for B200, as a thin Python binding over libdgb200.so.
+
+Every function here only checks shapes/dtypes/devices on the host and passes
+raw pointers to the C ABI declared in ``include/dgb200.h``; all arithmetic runs
+in the library's CUDA kernels. There is no fallback: if the shared library is
+missing or cannot run on the current device, calls raise.
+
+Tensors are torch tensors used as device memory; work is queued on torch's
+current CUDA stream. No call synchronises or allocates (except the
+convenience allocations of ``pack_ue8m0`` / ``empty_*`` when no output is
+given), so the calls can be captured in a CUDA Graph.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
+    "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+    "pack_ue8m0", "pack_ue8m0_validate", "DgError",
+    "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
+]
+
+BLOCK = 128
+DEVERR_TIMEOUT = 1
+DEVERR_MIXED_EXPERT_BLOCK = 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libdgb200.so"
+_lib = None
+_lock = threading.Lock()
+
+_STATUS = {
+    0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_ALIGNMENT", 3: "DG_ERR_UNSUPPORTED",
+    4: "DG_ERR_NOT_INITIALIZED", 5: "DG_ERR_CUDA",
+}
+
+
+class DgError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)}")
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load():
+    """Load libdgb200.so (built in-tree) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m moe_grouped_gemm_tcgen05_b200.build`")
+        L = ctypes.CDLL(path)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.dgb200_status_string.restype = ctypes.c_char_p
+        L.dgb200_status_string.argtypes = [i32]
+        L.dgb200_init.restype = i32
+        L.dgb200_init.argtypes = []
+        L.dgb200_device_error.restype = i32
+        L.dgb200_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
+        L.dgb200_set_block_n.restype = i32
+        L.dgb200_set_block_n.argtypes = [i32]
+        L.dgb200_block_n_supported.restype = i32
+        L.dgb200_block_n_supported.argtypes = [i32]
+        L.fp8_gemm_nt.restype = i32
+        L.fp8_gemm_nt.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
+        L.m_grouped_fp8_gemm_nt_contiguous.restype = i32
+        L.m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.m_grouped_fp8_gemm_nt_masked.restype = i32
+        L.m_grouped_fp8_gemm_nt_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.pack_ue8m0.restype = i32
+        L.pack_ue8m0.argtypes = [vp, vp, i64, i32, vp]
+        L.pack_ue8m0_validate.restype = i32
+        L.pack_ue8m0_validate.argtypes = [vp, i64, i32, vp, vp]
+        _lib = L
+        return L
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise DgError(fn, status)
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtypes, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+_FP8 = (torch.float8_e4m3fn, torch.uint8)
+_I32 = (torch.int32,)
+_BF16 = (torch.bfloat16,)
+
+
+def init():
+    """Configure the kernels for the current device (do it before graph capture)."""
+    _check("dgb200_init", load().dgb200_init())
+
+
+def device_error(clear: bool = True) -> int:
+    """Device status bits (DEVERR_*); synchronises the device."""
+    v = ctypes.c_uint32(0)
+    _check("dgb200_device_error", load().dgb200_device_error(ctypes.byref(v), 1 if clear else 0))
+    return int(v.value)
+
+
+def set_block_n(block_n: int):
+    """Force the N tile width (0 = heuristic). For tests and tuning."""
+    _check("dgb200_set_block_n", load().dgb200_set_block_n(int(block_n)))
+
+
+def block_n_supported(block_n: int) -> bool:
+    return bool(load().dgb200_block_n_supported(int(block_n)))
+
+
+def _kp(K: int) -> int:
+    return (K // BLOCK + 3) // 4
+
+
+def fp8_gemm_nt(a, sfa, b, sfb, d):
+    """d[M, N] (bf16) = (a . sfa) @ (b . sfb)^T for E4M3 a [M, K], b [N, K]."""
+    _need(a, "a", _FP8)
+    M, K = a.shape
+    _need(b, "b", _FP8)
+    N = b.shape[0]
+    _need(b, "b", _FP8, (N, K))
+    _need(sfa, "sfa", _I32, (M, _kp(K)))
+    _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (M, N))
+    _check("fp8_gemm_nt", load().fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, d, m_indices):
+    """Contiguous M-grouped GEMM; rows tagged by expert in m_indices (-1 = padding)."""
+    _need(a, "a", _FP8)
+    M_total, K = a.shape
+    _need(b, "b", _FP8)
+    G, N = b.shape[0], b.shape[1]
+    _need(b, "b", _FP8, (G, N, K))
+    _need(sfa, "sfa", _I32, (M_total, _kp(K)))
+    _need(sfb, "sfb", _I32, (G, (N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (M_total, N))
+    _need(m_indices, "m_indices", _I32, (M_total,))
+    _check("m_grouped_fp8_gemm_nt_contiguous",
+           load().m_grouped_fp8_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(m_indices),
+                                                   M_total, N, K, G, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, max_m=None):
+    """Masked M-grouped GEMM; group g uses its first masked_m[g] rows (device tensor)."""
+    _need(a, "a", _FP8)
+    G, mm, K = a.shape
+    if max_m is None:
+        max_m = mm
+    if max_m != mm:
+        raise ValueError(f"max_m={max_m} does not match a.shape[1]={mm}")
+    _need(b, "b", _FP8)
+    N = b.shape[1]
+    _need(b, "b", _FP8, (G, N, K))
+    _need(sfa, "sfa", _I32, (G, max_m, _kp(K)))
+    _need(sfb, "sfb", _I32, (G, (N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (G, max_m, N))
+    _need(masked_m, "masked_m", _I32, (G,))
+    _check("m_grouped_fp8_gemm_nt_masked",
+           load().m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m),
+                                               G, max_m, N, K, _stream()))
+    return d
+
+
+def pack_ue8m0(sf, out=None):
+    """Pack fp32 scales [..., cols] into int32 [..., ceil(cols/4)] (UE8M0, 4 per word)."""
+    _need(sf, "sf", (torch.float32,))
+    if sf.dim() < 1:
+        raise ValueError("sf must have at least one dimension")
+    cols = sf.shape[-1]
+    rows = sf.numel() // cols if cols else 0
+    kp = (cols + 3) // 4
+    if out is None:
+        out = torch.empty((*sf.shape[:-1], kp), dtype=torch.int32, device=sf.device)
+    _need(out, "out", _I32, (*sf.shape[:-1], kp))
+    _check("pack_ue8m0", load().pack_ue8m0(_ptr(sf), _ptr(out), rows, cols, _stream()))
+    return out
+
+
+def pack_ue8m0_validate(sf, bad_count):
+    """Write to bad_count (device int32 [1]) the number of scales with sign set or mantissa != 0."""
+    _need(sf, "sf", (torch.float32,))
+    _need(bad_count, "bad_count", _I32, (1,))
+    cols = sf.shape[-1]
+    rows = sf.numel() // cols if cols else 0
+    _check("pack_ue8m0_validate", load().pack_ue8m0_validate(_ptr(sf), rows, cols, _ptr(bad_count), _stream()))
+    return bad_count

@@ -1,0 +1,350 @@
+// Host side of libdgb200.so: the C ABI declared in include/dgb200.h.
+//
+// Each compute call validates its scalars and pointers on the host, encodes
+// the TMA tensor maps (driver entry point, no libcuda link), picks a tile
+// width from the sizes and the SM count, and launches one kernel on the
+// caller's stream. Nothing here allocates device memory, synchronises, or reads
+// a device value, so every compute call can be captured in a CUDA Graph.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "dgb200.h"
+#include "gemm_kernel.cuh"
+#include "pack_kernel.cuh"
+
+// Device status word (DG_DEVERR_* bits). One per device that loads the library.
+__device__ uint32_t g_dg_device_status = 0;
+
+namespace {
+
+using dg::GemmParams;
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    int sms = 0;
+    uint32_t* status = nullptr;  // address of g_dg_device_status on this device
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_force_bn{0};
+
+// --------------------------------------------------------------- kernels ----
+
+template <int BN, int KIND>
+void* kernel_ptr() {
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND>);
+}
+
+struct KernelEntry {
+    int bn;
+    int kind;
+    void* fn;
+    int smem;
+};
+
+#define DG_ENTRY(BN, KIND) {BN, KIND, kernel_ptr<BN, KIND>(), dg::GemmConfig<BN>::SMEM_BYTES}
+#define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense), DG_ENTRY(BN, dg::kContiguous), DG_ENTRY(BN, dg::kMasked)
+
+const KernelEntry kKernels[] = {
+    DG_ALL_KINDS(64), DG_ALL_KINDS(128), DG_ALL_KINDS(176), DG_ALL_KINDS(224), DG_ALL_KINDS(256),
+};
+constexpr int kBlockNs[] = {64, 128, 176, 224, 256};
+
+const KernelEntry* find_kernel(int bn, int kind) {
+    for (const auto& e : kKernels)
+        if (e.bn == bn && e.kind == kind) return &e;
+    return nullptr;
+}
+
+// ------------------------------------------------------------------ init ----
+
+dg_status init_device(int dev) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    DeviceState& st = g_dev[dev];
+    if (st.ready) return DG_OK;
+    if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return DG_ERR_NOT_INITIALIZED;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+        return DG_ERR_CUDA;
+    if (major != 10 || minor != 0) return DG_ERR_UNSUPPORTED;  // built for sm_100a only
+    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
+    for (const auto& e : kKernels) {
+        if (cudaFuncSetAttribute(e.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, e.smem) != cudaSuccess)
+            return DG_ERR_CUDA;
+    }
+    void* status = nullptr;
+    if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
+    st.status = static_cast<uint32_t*>(status);
+    st.ready = true;
+    return DG_OK;
+}
+
+dg_status current_device(DeviceState** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    if (!g_dev[dev].ready) {
+        dg_status s = init_device(dev);
+        if (s != DG_OK) return s;
+    }
+    *out = &g_dev[dev];
+    return DG_OK;
+}
+
+// ------------------------------------------------------------ tensor maps --
+
+bool encode_kmajor_u8(CUtensorMap* map, const void* base, int rank, uint64_t k, uint64_t rows, uint64_t mats,
+                      uint32_t box_rows) {
+    cuuint64_t dims[3] = {k, rows, mats};
+    cuuint64_t strides[2] = {k, k * rows};  // bytes, dims 1..rank-1
+    cuuint32_t box[3] = {128, box_rows, 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                          dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------- heuristics --
+
+// Time of one K=32 MMA step of a 128 x bn tile in tensor-pipe clocks: the
+// tensor core needs bn/2 clocks, and shared memory must deliver the A (4 KB)
+// and B (32*bn bytes) slices at about 128 bytes per clock.
+double mma_step_clocks(int bn) {
+    const double tc = bn / 2.0;
+    const double sm = (4096.0 + 32.0 * bn) / 128.0;
+    return tc > sm ? tc : sm;
+}
+
+int choose_block_n(long long m_blocks, int n, int sms) {
+    const int forced = g_force_bn.load();
+    if (forced != 0) return forced;
+    int best = 128;
+    double best_cost = 1e300;
+    for (int bn : kBlockNs) {
+        const long long nb = (n + bn - 1) / bn;
+        const long long tiles = m_blocks * nb;
+        const long long waves = (tiles + sms - 1) / sms;
+        // work in the last partial N tile is wasted in proportion to its empty columns
+        const double cost = static_cast<double>(waves) * mma_step_clocks(bn);
+        if (cost < best_cost * 0.999 || (cost <= best_cost * 1.001 && bn > best)) {
+            best_cost = cost;
+            best = bn;
+        }
+    }
+    return best;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+dg_status check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* d, int N,
+                       int K) {
+    if (!a || !sfa || !b || !sfb || !d) return DG_ERR_INVALID_ARG;
+    if (N <= 0 || K <= 0) return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N % 8 != 0) return DG_ERR_INVALID_ARG;
+    if (K > (1 << 20)) return DG_ERR_UNSUPPORTED;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(sfa, 4) || !aligned(sfb, 4))
+        return DG_ERR_ALIGNMENT;
+    return DG_OK;
+}
+
+dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
+                      void* stream, DeviceState* st, const void* a, const void* b, int a_rank, int b_rank,
+                      uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
+    const int bn = choose_block_n(m_blocks_for_heuristic, p.n, st->sms);
+    const KernelEntry* e = find_kernel(bn, kind);
+    if (e == nullptr) return DG_ERR_UNSUPPORTED;
+    p.status = st->status;
+    p.kb = p.k / 128;
+    p.kp = (p.kb + 3) / 4;
+    p.nb_sf = (p.n + 127) / 128;
+    p.num_n_blocks = (p.n + bn - 1) / bn;
+    p.raster_group = 16;
+    if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
+    if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn)))
+        return DG_ERR_INVALID_ARG;
+    const long long tiles = max_tiles_per_nblock * p.num_n_blocks;
+    if (tiles <= 0) return DG_OK;
+    const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+    void* args[] = {&p};
+    cudaError_t err = cudaLaunchKernel(e->fn, dim3(grid), dim3(dg::NUM_THREADS), args, static_cast<size_t>(e->smem),
+                                       static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dgb200_status_string(dg_status s) {
+    switch (s) {
+        case DG_OK: return "DG_OK";
+        case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+        case DG_ERR_ALIGNMENT: return "DG_ERR_ALIGNMENT";
+        case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
+        case DG_ERR_NOT_INITIALIZED: return "DG_ERR_NOT_INITIALIZED";
+        case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    }
+    return "DG_ERR_UNKNOWN";
+}
+
+dg_status dgb200_init(void) {
+    DeviceState* st = nullptr;
+    return current_device(&st);
+}
+
+dg_status dgb200_device_error(uint32_t* bits, int clear) {
+    if (bits == nullptr) return DG_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    dg_status s = current_device(&st);
+    if (s != DG_OK) return s;
+    if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
+    if (cudaMemcpy(bits, st->status, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
+    if (clear && cudaMemset(st->status, 0, sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+    return DG_OK;
+}
+
+int dgb200_block_n_supported(int block_n) {
+    for (int bn : kBlockNs)
+        if (bn == block_n) return 1;
+    return 0;
+}
+
+dg_status dgb200_set_block_n(int block_n) {
+    if (block_n != 0 && !dgb200_block_n_supported(block_n)) return DG_ERR_UNSUPPORTED;
+    g_force_bn.store(block_n);
+    return DG_OK;
+}
+
+dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
+                      int K, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M <= 0) return DG_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = nullptr;
+    p.rows = M;
+    p.n = N;
+    p.k = K;
+    p.groups = 1;
+    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
+    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, stream, st, a, b, 2, 2,
+                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+}
+
+dg_status m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                           void* d, const int32_t* m_indices, int M_total, int N, int K, int G,
+                                           void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M_total <= 0 || G <= 0 || m_indices == nullptr) return DG_ERR_INVALID_ARG;
+    if (!aligned(m_indices, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = m_indices;
+    p.rows = M_total;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (M_total + dg::BM - 1) / dg::BM;
+    return launch_gemm(dg::kContiguous, p, p.num_m_blocks, p.num_m_blocks, stream, st, a, b, 2, 3,
+                       static_cast<uint64_t>(M_total), 1, static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+}
+
+dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                                       const int32_t* masked_m, int G, int max_m, int N, int K, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (G <= 0 || max_m <= 0 || masked_m == nullptr) return DG_ERR_INVALID_ARG;
+    if (G > dg::MAX_MASKED_GROUPS) return DG_ERR_UNSUPPORTED;
+    if (!aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = masked_m;
+    p.rows = max_m;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (max_m + dg::BM - 1) / dg::BM;
+    const long long mb_total = static_cast<long long>(G) * p.num_m_blocks;
+    return launch_gemm(dg::kMasked, p, mb_total, mb_total, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
+                       static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+}
+
+dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int cols, void* stream) {
+    if (!sf || !packed || rows <= 0 || cols <= 0) return DG_ERR_INVALID_ARG;
+    if (!aligned(sf, 4) || !aligned(packed, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    dg_status s = current_device(&st);
+    if (s != DG_OK) return s;
+    const int kp = (cols + 3) / 4;
+    const int64_t words = rows * kp;
+    const int threads = 256;
+    int64_t blocks = (words + threads - 1) / threads;
+    const int64_t cap = static_cast<int64_t>(st->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cols % 4 == 0 && aligned(sf, 16)) {
+        dg::pack_ue8m0_vec4_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(
+            reinterpret_cast<const float4*>(sf), reinterpret_cast<uint32_t*>(packed), words);
+    } else {
+        dg::pack_ue8m0_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(
+            sf, reinterpret_cast<uint32_t*>(packed), rows, cols, kp);
+    }
+    return cudaPeekAtLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* bad_count, void* stream) {
+    if (!sf || !bad_count || rows <= 0 || cols <= 0) return DG_ERR_INVALID_ARG;
+    if (!aligned(sf, 4) || !aligned(bad_count, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    dg_status s = current_device(&st);
+    if (s != DG_OK) return s;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(bad_count, 0, sizeof(int32_t), cs) != cudaSuccess) return DG_ERR_CUDA;
+    const int64_t n = rows * cols;
+    const int threads = 256;
+    int64_t blocks = (n + threads - 1) / threads;
+    const int64_t cap = static_cast<int64_t>(st->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    dg::pack_ue8m0_validate_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(sf, n, bad_count);
+    return cudaPeekAtLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
+}  // extern "C"

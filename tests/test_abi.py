@@ -1,0 +1,78 @@
+"""The C-ABI library builds, loads and exports every declared symbol; host-side
+argument checks reject bad calls before any device work (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_grouped_gemm_tcgen05_b200 as dg
+from moe_grouped_gemm_tcgen05_b200 import build as dgbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dgb200.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"DG_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dgbuild.build()
+    return ctypes.CDLL(dgbuild.LIB)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ("fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
+              "pack_ue8m0", "pack_ue8m0_validate", "dgb200_init", "dgb200_device_error"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    lib.dgb200_status_string.restype = ctypes.c_char_p
+    assert lib.dgb200_status_string(0) == b"DG_OK"
+    assert lib.dgb200_status_string(1) == b"DG_ERR_INVALID_ARG"
+    assert lib.dgb200_status_string(5) == b"DG_ERR_CUDA"
+
+
+def test_host_argument_checks_fail_before_device_work(lib):
+    vp = ctypes.c_void_p
+    f = lib.fp8_gemm_nt
+    f.restype = ctypes.c_int
+    f.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+    good = vp(0x10000)
+    assert f(None, good, good, good, good, 128, 128, 128, None) == 1          # null pointer
+    assert f(good, good, good, good, good, 128, 128, 100, None) == 1          # K % 128
+    assert f(good, good, good, good, good, 128, 12, 128, None) == 1           # N % 8
+    assert f(good, good, good, good, good, 0, 128, 128, None) == 1            # M <= 0
+    assert f(vp(0x10004), good, good, good, good, 128, 128, 128, None) == 2   # A alignment
+    m = lib.m_grouped_fp8_gemm_nt_masked
+    m.restype = ctypes.c_int
+    m.argtypes = [vp] * 6 + [ctypes.c_int] * 4 + [vp]
+    assert m(good, good, good, good, good, None, 4, 64, 128, 128, None) == 1  # null masked_m
+    assert m(good, good, good, good, good, good, 2048, 64, 128, 128, None) == 3  # too many groups
+    p = lib.pack_ue8m0
+    p.restype = ctypes.c_int
+    p.argtypes = [vp, vp, ctypes.c_int64, ctypes.c_int, vp]
+    assert p(None, good, 4, 4, None) == 1
+    assert p(good, good, 0, 4, None) == 1
+    assert p(vp(0x10002), good, 4, 4, None) == 2
+
+
+def test_binding_fails_loudly_without_cuda():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    a = torch.zeros((128, 128), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        dg.fp8_gemm_nt(a, torch.zeros((128, 1), dtype=torch.int32), a,
+                       torch.zeros((1, 1), dtype=torch.int32), torch.zeros((128, 128), dtype=torch.bfloat16))

@@ -1,0 +1,219 @@
+"""GEMM parity on the GPU vs the CPU oracle at sizes the oracle finishes in
+seconds: several tiles, ragged M/N/K tails, every tile width, exact one-hot
+cases, masked and contiguous forms with sentinel-checked untouched rows, and
+CUDA Graph replay with new masked_m. All calls go through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import moe_grouped_gemm_tcgen05_b200 as dg
+from moe_grouped_gemm_tcgen05_b200 import workloads as W
+
+from helpers import bf16_to_f64, check_fp, fill_sentinel, is_sentinel
+
+pytestmark = pytest.mark.gpu
+
+BLOCK_NS = [64, 128, 176, 224, 256]
+
+
+@pytest.fixture(autouse=True)
+def _reset():
+    dg.init()
+    dg.device_error(clear=True)
+    yield
+    dg.set_block_n(0)
+    assert dg.device_error(clear=True) & dg.DEVERR_TIMEOUT == 0
+
+
+def _dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _pack_dev(sf_f32):
+    return dg.pack_ue8m0(_dev(sf_f32))
+
+
+def _oracle_pack(sf_f32):
+    return oracle.pack_ue8m0(sf_f32.reshape(-1, sf_f32.shape[-1])).reshape(*sf_f32.shape[:-1], -1)
+
+
+def run_dense(p, bn=0):
+    dg.set_block_n(bn)
+    d = torch.empty((p["M"], p["N"]), dtype=torch.bfloat16, device="cuda")
+    fill_sentinel(d)
+    dg.fp8_gemm_nt(_dev(p["a"]), _pack_dev(p["sfa_f32"]), _dev(p["b"]), _pack_dev(p["sfb_f32"]), d)
+    torch.cuda.synchronize()
+    return d
+
+
+def ref_dense(p):
+    return oracle.fp8_gemm_nt(p["a"], _oracle_pack(p["sfa_f32"]), p["b"], _oracle_pack(p["sfb_f32"]))
+
+
+@pytest.mark.parametrize("bn", BLOCK_NS)
+@pytest.mark.parametrize("mnk", [(128, 256, 512), (300, 400, 1024), (257, 264, 640)])
+def test_dense_parity_every_tile_width(bn, mnk):
+    p = W.dense(*mnk, seed=sum(mnk))
+    d = run_dense(p, bn)
+    assert not is_sentinel(d).any()
+    check_fp(bf16_to_f64(d), ref_dense(p), f"dense {mnk} bn={bn}")
+
+
+@pytest.mark.parametrize("mnk", [(1, 16, 128), (64, 2112, 896), (128, 8, 128), (513, 1000, 2048)])
+def test_dense_parity_edge_shapes(mnk):
+    p = W.dense(*mnk, seed=7)
+    d = run_dense(p)
+    check_fp(bf16_to_f64(d), ref_dense(p), f"dense {mnk}")
+
+
+def test_dense_workload0():
+    p = W.workload0()
+    check_fp(bf16_to_f64(run_dense(p)), ref_dense(p), "workload 0")
+
+
+def _codes(rng, shape):
+    s = rng.integers(0, 2, size=shape)
+    e = rng.integers(4, 12, size=shape)
+    m = rng.integers(0, 8, size=shape)
+    return ((s << 7) | (e << 3) | m).astype(np.uint8)
+
+
+def _pack_bytes_host(byts):
+    rows, cols = byts.shape
+    kp = (cols + 3) // 4
+    w = np.zeros((rows, kp), dtype=np.int64)
+    for c in range(cols):
+        w[:, c // 4] |= byts[:, c].astype(np.int64) << (8 * (c % 4))
+    return w.astype(np.uint32).view(np.int32)
+
+
+@pytest.mark.parametrize("bn", BLOCK_NS)
+def test_one_hot_rows_are_bit_exact(bn):
+    # one-hot A rows with power-of-two scales: every output is a single product
+    # e4m3 * 2^a * 2^b, exactly representable in bf16
+    rng = np.random.default_rng(bn)
+    M, N, K = 200, 304, 1152
+    KB = K // 128
+    ks = rng.integers(0, K, size=M)
+    a = np.zeros((M, K), dtype=np.uint8)
+    a[np.arange(M), ks] = 0x38
+    ea = rng.integers(120, 134, size=(M, KB)).astype(np.uint8)
+    eb = rng.integers(120, 134, size=(3, KB)).astype(np.uint8)
+    b = _codes(rng, (N, K))
+    sfa, sfb = _pack_bytes_host(ea), _pack_bytes_host(eb)
+    dg.set_block_n(bn)
+    d = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    dg.fp8_gemm_nt(_dev(a), _dev(sfa), _dev(b), _dev(sfb), d)
+    want = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    want_bf16 = torch.from_numpy(want).to(torch.bfloat16)
+    assert torch.equal(torch.from_numpy(want_bf16.to(torch.float64).numpy()), torch.from_numpy(want)), "not exact in bf16"
+    assert torch.equal(d.cpu().view(torch.int16), want_bf16.view(torch.int16))
+
+
+# ------------------------------------------------------------------ masked --
+
+def run_masked(p, masked_m=None, bn=0):
+    dg.set_block_n(bn)
+    G, max_m, N = p["G"], p["max_m"], p["N"]
+    d = fill_sentinel(torch.empty((G, max_m, N), dtype=torch.bfloat16, device="cuda"))
+    mm = p["masked_m"] if masked_m is None else masked_m
+    dg.m_grouped_fp8_gemm_nt_masked(_dev(p["a"]), _pack_dev(p["sfa_f32"]), _dev(p["b"]), _pack_dev(p["sfb_f32"]),
+                                    d, _dev(np.asarray(mm, dtype=np.int32)))
+    torch.cuda.synchronize()
+    return d
+
+
+def check_masked(p, d, masked_m=None, what="masked"):
+    mm = p["masked_m"] if masked_m is None else masked_m
+    ref, valid = oracle.m_grouped_fp8_gemm_nt_masked(p["a"], _oracle_pack(p["sfa_f32"]), p["b"],
+                                                     _oracle_pack(p["sfb_f32"]), mm)
+    sent = is_sentinel(d)
+    assert sent[~valid].all(), f"{what}: a row past masked_m was written"
+    assert not sent[valid].any(), f"{what}: a valid row was not written"
+    check_fp(bf16_to_f64(d)[valid], ref[valid], what)
+
+
+@pytest.mark.parametrize("bn", [64, 128, 176, 256])
+def test_masked_parity_and_sentinel(bn):
+    mm = np.array([0, 1, 128, 200, 77, -3, 500], dtype=np.int32)
+    p = W.masked(mm, 200, 272, 384, seed=11)
+    d = run_masked(p, bn=bn)
+    check_masked(p, d, what=f"masked bn={bn}")
+
+
+def test_masked_all_empty_writes_nothing():
+    p = W.masked(np.zeros(4, dtype=np.int32), 64, 128, 256, seed=12)
+    d = run_masked(p)
+    assert is_sentinel(d).all()
+
+
+def test_masked_graph_replay_with_new_masked_m():
+    G, max_m, N, K = 6, 256, 384, 512
+    p = W.masked(np.full(G, max_m, dtype=np.int32), max_m, N, K, seed=13, fill_invalid_nan=False)
+    a, b = _dev(p["a"]), _dev(p["b"])
+    sfa, sfb = _pack_dev(p["sfa_f32"]), _pack_dev(p["sfb_f32"])
+    mm_dev = torch.zeros(G, dtype=torch.int32, device="cuda")
+    d = torch.empty((G, max_m, N), dtype=torch.bfloat16, device="cuda")
+    dg.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, mm_dev)  # warm-up before capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dg.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, mm_dev)
+    rng = np.random.default_rng(5)
+    for it in range(3):
+        new = rng.integers(0, max_m + 1, size=G).astype(np.int32)
+        new[it] = 0
+        mm_dev.copy_(torch.from_numpy(new))
+        fill_sentinel(d)
+        g.replay()
+        torch.cuda.synchronize()
+        check_masked(p, d, masked_m=new, what=f"replay {it}")
+    del g
+
+
+# -------------------------------------------------------------- contiguous --
+
+def run_contig(p, m_indices=None, bn=0):
+    dg.set_block_n(bn)
+    mi = p["m_indices"] if m_indices is None else m_indices
+    d = fill_sentinel(torch.empty((p["M_total"], p["N"]), dtype=torch.bfloat16, device="cuda"))
+    dg.m_grouped_fp8_gemm_nt_contiguous(_dev(p["a"]), _pack_dev(p["sfa_f32"]), _dev(p["b"]),
+                                        _pack_dev(p["sfb_f32"]), d, _dev(mi))
+    torch.cuda.synchronize()
+    return d
+
+
+def check_contig(p, d, m_indices=None, what="contiguous"):
+    mi = p["m_indices"] if m_indices is None else m_indices
+    ref, valid = oracle.m_grouped_fp8_gemm_nt_contiguous(p["a"], _oracle_pack(p["sfa_f32"]), p["b"],
+                                                         _oracle_pack(p["sfb_f32"]), mi)
+    sent = is_sentinel(d)
+    assert sent[~valid].all(), f"{what}: a padding row was written"
+    assert not sent[valid].any(), f"{what}: a valid row was not written"
+    check_fp(bf16_to_f64(d)[valid], ref[valid], what)
+
+
+@pytest.mark.parametrize("bn", [64, 128, 224, 256])
+def test_contiguous_parity_and_padding(bn):
+    p = W.contiguous([5, 0, 130, 128, 1], 264, 512, seed=21, tail_blocks=1)
+    d = run_contig(p, bn=bn)
+    check_contig(p, d, what=f"contiguous bn={bn}")
+    assert dg.device_error(clear=True) == 0
+
+
+def test_contiguous_mixed_block_is_flagged():
+    p = W.contiguous([100, 100], 128, 256, seed=22)
+    mi = p["m_indices"].copy()
+    mi[40:60] = 1  # expert 1 inside expert 0's first block
+    d = run_contig(p, m_indices=mi)
+    assert dg.device_error(clear=True) & dg.DEVERR_MIXED_EXPERT_BLOCK
+    # the block's rows of the larger index are computed, the others untouched
+    sent = is_sentinel(d)
+    assert sent[0:40].all() and sent[60:128].all()
+    ref, _ = oracle.m_grouped_fp8_gemm_nt_contiguous(p["a"], _oracle_pack(p["sfa_f32"]), p["b"],
+                                                     _oracle_pack(p["sfb_f32"]), mi)
+    check_fp(bf16_to_f64(d)[40:60], ref[40:60], "mixed block rows")
+    ok = np.nonzero(mi[128:] >= 0)[0] + 128
+    check_fp(bf16_to_f64(d)[ok], ref[ok], "clean blocks")
