@@ -105,6 +105,16 @@ DG_API dg_status dgb200_set_block_n(int block_n);
 DG_API int dgb200_block_n_supported(int block_n);
 
 /*
+ * Test hook for the failure path (process-wide). wait_limit_ms bounds every
+ * wait inside the GEMM kernels (0 restores the default, 2000 ms). mode 1 makes
+ * CTA 0 of each GEMM launch withhold the arrive of its first pipeline stage,
+ * so a wait runs out: that launch leaves its output incomplete, sets
+ * DG_DEVERR_TIMEOUT and returns; the CUDA context stays usable. mode 0 is
+ * normal operation.
+ */
+DG_API dg_status dgb200_set_test_hooks(int mode, int wait_limit_ms);
+
+/*
  * Dense FP8 NT GEMM ("DeepInside DeepGEMM", section 4: fp8_gemm_nt).
  *   a   : device, E4M3 [M, K]
  *   sfa : device, int32 [M, KP]             packed UE8M0, one per 1x128 block

@@ -38,6 +38,8 @@ std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_bn{0};
+std::atomic<int> g_test_mode{0};
+std::atomic<uint64_t> g_wait_limit_ns{dg::DEFAULT_WAIT_LIMIT_NS};
 
 // --------------------------------------------------------------- kernels ----
 
@@ -180,6 +182,8 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     p.nb_sf = (p.n + 127) / 128;
     p.num_n_blocks = (p.n + bn - 1) / bn;
     p.raster_group = 16;
+    p.wait_limit_ns = g_wait_limit_ns.load();
+    p.test_mode = g_test_mode.load();
     if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
     if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn)))
         return DG_ERR_INVALID_ARG;
@@ -233,6 +237,14 @@ int dgb200_block_n_supported(int block_n) {
 dg_status dgb200_set_block_n(int block_n) {
     if (block_n != 0 && !dgb200_block_n_supported(block_n)) return DG_ERR_UNSUPPORTED;
     g_force_bn.store(block_n);
+    return DG_OK;
+}
+
+dg_status dgb200_set_test_hooks(int mode, int wait_limit_ms) {
+    if (mode < 0 || mode > 1 || wait_limit_ms < 0) return DG_ERR_INVALID_ARG;
+    g_test_mode.store(mode);
+    g_wait_limit_ns.store(wait_limit_ms == 0 ? dg::DEFAULT_WAIT_LIMIT_NS
+                                             : static_cast<uint64_t>(wait_limit_ms) * 1000000ull);
     return DG_OK;
 }
 

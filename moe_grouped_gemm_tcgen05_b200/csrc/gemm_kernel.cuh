@@ -50,7 +50,7 @@ constexpr int MMA_K = 32;               // K of one kind::mxf8f6f4 MMA
 constexpr int NUM_THREADS = 192;
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
-constexpr long long WAIT_LIMIT_CYCLES = 4000000000LL;  // ~2 s
+constexpr uint64_t DEFAULT_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 
 constexpr uint32_t DEVERR_TIMEOUT = 1u;
 constexpr uint32_t DEVERR_MIXED_EXPERT_BLOCK = 2u;
@@ -71,6 +71,8 @@ struct GemmParams {
     int num_m_blocks;         // ceil(rows / 128)
     int num_n_blocks;         // ceil(N / BN)
     int raster_group;         // m-blocks per raster band (dense / contiguous)
+    uint64_t wait_limit_ns;   // bound of every mbarrier wait
+    int test_mode;            // 1: CTA 0 withholds one stage arrive (exercises the timeout path)
 };
 
 template <int BN>
@@ -105,18 +107,34 @@ struct Tile {
 
 // ----------------------------------------------------------------- waits ----
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of `bar` with the given parity. Gives up when another
+// role of this CTA has given up, or after p.wait_limit_ns; a timeout is
+// recorded in the device status word.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const GemmParams& p,
                                              volatile int* s_abort) {
     if (mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
+    const uint64_t t0 = global_ns();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*s_abort) return false;
-        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+        if (global_ns() - t0 > p.wait_limit_ns) {
             atomicOr(p.status, DEVERR_TIMEOUT);
             *s_abort = 1;
             return false;
         }
+    }
+}
+
+// Bounded wait used only while unwinding: no status update.
+__device__ __forceinline__ void wait_quiet(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity) && global_ns() - t0 < limit_ns) {
     }
 }
 
@@ -356,7 +374,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     sw.store(smem_sfa + stage * Cfg::SFA_BYTES, smem_sfb + stage * Cfg::SFB_BYTES, lane);
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&full_bar[stage]);
+                    // test hook: CTA 0 withholds the arrive of its first stage
+                    const bool withhold = p.test_mode == 1 && blockIdx.x == 0 && issued == 0;
+                    if (lane == 0 && !withhold) mbar_arrive(&full_bar[stage]);
                     // start the loads of the following group
                     if (ahead_ok) {
                         if (++ahead_kg == kg_count) {
@@ -380,8 +400,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             uint32_t ph = phase;
             for (int i = 0; i < STAGES && i < issued; ++i) {
                 if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
-                const long long t0 = clock64();
-                while (!mbar_try_wait(&full_bar[s], ph) && clock64() - t0 < WAIT_LIMIT_CYCLES / 64) {}
+                wait_quiet(&full_bar[s], ph, p.wait_limit_ns / 16);
             }
         }
     } else if (warp == 1) {
@@ -436,10 +455,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         // all MMAs of this CTA must finish before TMEM is released
         if (lane == 0) tc_commit(drain_bar);
         __syncwarp();
-        {
-            const long long t0 = clock64();
-            while (!mbar_try_wait(drain_bar, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
-        }
+        wait_quiet(drain_bar, 0, p.wait_limit_ns);
     } else {
         // ------------------------------------------------------- epilogue --
         const int q = static_cast<int>(warp & 3);   // TMEM sub-partition of this warp

@@ -181,3 +181,105 @@ def zipf_masked_m(rng, G: int = 256, max_m: int = 512, a: float = 1.1):
 def workload4():
     mm = zipf_masked_m(rng_for(1004))
     return masked(mm, 512, 7168, 2048, seed=1004, fill_invalid_nan=False)
+
+
+# ---- device-side generation for full-size workloads ------------------------
+#
+# Same recipe as above (N(0,1) draws, power-of-two block scales from the block
+# amax, E4M3 round-to-nearest-even), drawn with torch's seeded generator on the
+# target device so that multi-GB weights are produced in milliseconds. The
+# random stream differs from numpy's; tests that use these inputs copy them to
+# the host for the oracle.
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _pow2_scale_t(amax: torch.Tensor) -> torch.Tensor:
+    v = amax.to(torch.float64).clamp_min(AMAX_FLOOR) / E4M3_MAX
+    mant, exp = torch.frexp(v)
+    e = torch.where(mant == 0.5, exp - 1, exp)
+    return torch.ldexp(torch.ones_like(v), e).to(torch.float32)
+
+
+def quantise_rows_t(x: torch.Tensor):
+    """x float32 [R, K] (any device) -> (uint8 [R, K], float32 [R, K/128])."""
+    R, K = x.shape
+    xb = x.view(R, K // BLOCK, BLOCK)
+    s = _pow2_scale_t(xb.abs().amax(dim=2))
+    q = (xb / s[:, :, None]).to(torch.float8_e4m3fn).view(torch.uint8).reshape(R, K)
+    return q, s
+
+
+def quantise_blocks_t(w: torch.Tensor):
+    """w float32 [N, K] -> (uint8 [N, K], float32 [ceil(N/128), K/128])."""
+    N, K = w.shape
+    NB = (N + BLOCK - 1) // BLOCK
+    if NB * BLOCK != N:
+        w = torch.cat([w, torch.zeros((NB * BLOCK - N, K), dtype=w.dtype, device=w.device)])
+    wb = w.view(NB, BLOCK, K // BLOCK, BLOCK)
+    s = _pow2_scale_t(wb.abs().amax(dim=(1, 3)))
+    q = (wb / s[:, None, :, None]).to(torch.float8_e4m3fn).view(torch.uint8).reshape(NB * BLOCK, K)[:N]
+    return q.contiguous(), s
+
+
+def dense_t(M: int, N: int, K: int, seed: int, device="cuda"):
+    g = _gen(device, seed)
+    a, sfa = quantise_rows_t(torch.randn((M, K), generator=g, device=device))
+    b, sfb = quantise_blocks_t(torch.randn((N, K), generator=g, device=device))
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, M=M, N=N, K=K)
+
+
+def grouped_weights_t(g, G: int, N: int, K: int, device):
+    NB = (N + BLOCK - 1) // BLOCK
+    b = torch.empty((G, N, K), dtype=torch.uint8, device=device)
+    sfb = torch.empty((G, NB, K // BLOCK), dtype=torch.float32, device=device)
+    for i in range(G):
+        b[i], sfb[i] = quantise_blocks_t(torch.randn((N, K), generator=g, device=device))
+    return b, sfb
+
+
+def contiguous_t(counts, N: int, K: int, seed: int, align: int = BLOCK, device="cuda"):
+    G = len(counts)
+    seg = [((int(c) + align - 1) // align) * align for c in counts]
+    M_total = int(sum(seg))
+    mi = np.full(M_total, -1, dtype=np.int32)
+    off = 0
+    for e, (c, s) in enumerate(zip(counts, seg)):
+        mi[off:off + int(c)] = e
+        off += s
+    g = _gen(device, seed)
+    a, sfa = quantise_rows_t(torch.randn((M_total, K), generator=g, device=device))
+    b, sfb = grouped_weights_t(g, G, N, K, device)
+    m_indices = torch.from_numpy(mi).to(device)
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, m_indices=m_indices, M_total=M_total, N=N, K=K, G=G)
+
+
+def masked_t(masked_m, max_m: int, N: int, K: int, seed: int, device="cuda"):
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = masked_m.shape[0]
+    g = _gen(device, seed)
+    a, sfa = quantise_rows_t(torch.randn((G * max_m, K), generator=g, device=device))
+    b, sfb = grouped_weights_t(g, G, N, K, device)
+    return dict(a=a.view(G, max_m, K), sfa_f32=sfa.view(G, max_m, K // BLOCK), b=b, sfb_f32=sfb,
+                masked_m=torch.from_numpy(masked_m).to(device), masked_m_host=masked_m,
+                G=G, max_m=max_m, N=N, K=K)
+
+
+def workload1_t(M: int, N: int, K: int, device="cuda"):
+    return dense_t(M, N, K, seed=1001 + 7 * M + N, device=device)
+
+
+def workload2_t(device="cuda"):
+    return contiguous_t(contiguous_counts(), 4096, 7168, seed=1002, device=device)
+
+
+def workload3_t(proj: str, device="cuda"):
+    N, K = (4096, 7168) if proj == "up" else (7168, 2048)
+    return masked_t(masked_m_uniform(rng_for(1003)), 256, N, K, seed=1003, device=device)
+
+
+def workload4_t(device="cuda"):
+    return masked_t(zipf_masked_m(rng_for(1004)), 512, 7168, 2048, seed=1004, device=device)

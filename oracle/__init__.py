@@ -39,6 +39,7 @@ from .gemm import (  # noqa: F401
     dequant_weights,
     fp8_gemm_nt,
     fp8_gemm_nt_sampled,
+    fp8_gemm_nt_points,
     m_grouped_fp8_gemm_nt_contiguous,
     m_grouped_fp8_gemm_nt_contiguous_sampled,
     m_grouped_fp8_gemm_nt_masked,

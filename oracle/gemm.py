@@ -161,3 +161,20 @@ def m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, groups, rows, cols):
         out[sel] = fp8_gemm_nt_sampled(np.asarray(a)[g], np.asarray(sfa)[g], np.asarray(b)[g],
                                        np.asarray(sfb)[g], rows[sel], cols[sel])
     return out
+
+
+def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb) -> np.ndarray:
+    """Outputs one at a time: out[i] = sum_k A^_i[k] * B^[n_idx[i], k].
+
+    a_rows / sfa_rows: the A rows of the sampled outputs and their packed scale
+    rows; b_rows: row n_idx[i] of B for each output; sfb: the full packed scale
+    matrix of that B ([ceil(N/128), KP]), indexed here by n_idx // 128.
+    """
+    A = dequant_rows(a_rows, sfa_rows)
+    b_rows = np.asarray(b_rows, dtype=np.uint8)
+    P, K = b_rows.shape
+    KB = _kb(K)
+    n_idx = np.asarray(n_idx, dtype=np.int64)
+    scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))[n_idx // BLOCK]
+    B = (e4m3_to_f64(b_rows).reshape(P, KB, BLOCK) * scale[:, :, None]).reshape(P, K)
+    return np.einsum("ik,ik->i", A, B)

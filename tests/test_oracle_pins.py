@@ -321,3 +321,17 @@ def _planted(kind):
 @pytest.mark.parametrize("kind", ["weight_scale_per_row", "byte_order_reversed", "transposed_b", "dropped_last_block"])
 def test_pins_catch_planted_mistakes(kind):
     assert not one_hot_check(_planted(kind)), kind
+
+
+def test_points_match_full():
+    rng = np.random.default_rng(8)
+    M, N, K = 9, 300, 640
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(rng.integers(120, 135, size=(M, 5)).astype(np.uint8))
+    sfb = _pack_bytes(rng.integers(120, 135, size=(3, 5)).astype(np.uint8))
+    full = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    r = rng.integers(0, M, size=40)
+    c = rng.integers(0, N, size=40)
+    pts = oracle.fp8_gemm_nt_points(a[r], sfa[r], b[c], c, sfb)
+    np.testing.assert_allclose(pts, full[r, c], rtol=1e-13, atol=0)
