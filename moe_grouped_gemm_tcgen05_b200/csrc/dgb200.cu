@@ -59,9 +59,10 @@ struct KernelEntry {
 #define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense), DG_ENTRY(BN, dg::kContiguous), DG_ENTRY(BN, dg::kMasked)
 
 const KernelEntry kKernels[] = {
-    DG_ALL_KINDS(64), DG_ALL_KINDS(128), DG_ALL_KINDS(176), DG_ALL_KINDS(224), DG_ALL_KINDS(256),
+    DG_ALL_KINDS(64),  DG_ALL_KINDS(96),  DG_ALL_KINDS(128), DG_ALL_KINDS(160),
+    DG_ALL_KINDS(192), DG_ALL_KINDS(224), DG_ALL_KINDS(256),
 };
-constexpr int kBlockNs[] = {64, 128, 176, 224, 256};
+constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
 
 const KernelEntry* find_kernel(int bn, int kind) {
     for (const auto& e : kKernels)
@@ -127,18 +128,42 @@ bool encode_kmajor_u8(CUtensorMap* map, const void* base, int rank, uint64_t k, 
     return r == CUDA_SUCCESS;
 }
 
-// ------------------------------------------------------------- heuristics --
-
-// Time of one K=32 MMA step of a 128 x bn tile in tensor-pipe clocks: the
-// tensor core needs bn/2 clocks, and shared memory must deliver the A (4 KB)
-// and B (32*bn bytes) slices at about 128 bytes per clock.
-double mma_step_clocks(int bn) {
-    const double tc = bn / 2.0;
-    const double sm = (4096.0 + 32.0 * bn) / 128.0;
-    return tc > sm ? tc : sm;
+// bf16 output, written by TMA in 32x32 boxes with the 64-byte swizzle.
+bool encode_d_bf16(CUtensorMap* map, void* base, int rank, uint64_t n, uint64_t rows, uint64_t mats) {
+    cuuint64_t dims[3] = {n, rows, mats};
+    cuuint64_t strides[2] = {2 * n, 2 * n * rows};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), base, dims, strides,
+                          box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
 }
 
-int choose_block_n(long long m_blocks, int n, int sms) {
+// ------------------------------------------------------------- heuristics --
+
+// Feed rate of one SM from L2 under full load, bytes per SM clock (from the
+// profile of the 4096x7168x16384 GEMM: ~700 clocks per 44 KB stage).
+constexpr double kL2BytesPerClk = 64.0;
+// Tensor-core clocks lost per tile when the accumulator is single-buffered
+// (the MMA warp waits for the epilogue's TMEM reads).
+constexpr double kSingleBufferBubble = 600.0;
+
+// Clocks one CTA spends per 128-K block of a (rows_a x bn) tile: the larger of
+// the tensor core (four K=32 MMAs of bn/2 clocks), shared-memory reads
+// (4 x (4 KB of A + 32*bn of B) at 128 B/clk) and the L2 feed of the stage.
+double kblock_clocks(int bn, int rows_a) {
+    const double tc = 2.0 * bn;
+    const double sm = 4.0 * (4096.0 + 32.0 * bn) / 128.0;
+    const double l2 = (rows_a + bn) * 128.0 / kL2BytesPerClk;
+    double t = tc > sm ? tc : sm;
+    return t > l2 ? t : l2;
+}
+
+int num_acc_for(int bn) { return (2 * bn + 4 + 4 * ((bn + 127) / 128) <= 512) ? 2 : 1; }
+
+// Pick the N tile with the least modelled time: waves of tiles x time per tile.
+int choose_block_n(long long m_blocks, int rows_a, int n, int kb, int sms) {
     const int forced = g_force_bn.load();
     if (forced != 0) return forced;
     int best = 128;
@@ -147,8 +172,8 @@ int choose_block_n(long long m_blocks, int n, int sms) {
         const long long nb = (n + bn - 1) / bn;
         const long long tiles = m_blocks * nb;
         const long long waves = (tiles + sms - 1) / sms;
-        // work in the last partial N tile is wasted in proportion to its empty columns
-        const double cost = static_cast<double>(waves) * mma_step_clocks(bn);
+        const double tile = kb * kblock_clocks(bn, rows_a) + (num_acc_for(bn) == 1 ? kSingleBufferBubble : 0.0);
+        const double cost = static_cast<double>(waves) * tile;
         if (cost < best_cost * 0.999 || (cost <= best_cost * 1.001 && bn > best)) {
             best_cost = cost;
             best = bn;
@@ -173,7 +198,8 @@ dg_status check_common(const void* a, const int32_t* sfa, const void* b, const i
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
                       void* stream, DeviceState* st, const void* a, const void* b, int a_rank, int b_rank,
                       uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
-    const int bn = choose_block_n(m_blocks_for_heuristic, p.n, st->sms);
+    const int rows_a = p.rows < dg::BM ? p.rows : dg::BM;
+    const int bn = choose_block_n(m_blocks_for_heuristic, rows_a, p.n, p.k / 128, st->sms);
     const KernelEntry* e = find_kernel(bn, kind);
     if (e == nullptr) return DG_ERR_UNSUPPORTED;
     p.status = st->status;
@@ -187,6 +213,7 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
     if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn)))
         return DG_ERR_INVALID_ARG;
+    if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
     const long long tiles = max_tiles_per_nblock * p.num_n_blocks;
     if (tiles <= 0) return DG_OK;
     const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);

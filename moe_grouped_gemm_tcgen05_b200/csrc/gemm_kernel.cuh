@@ -17,10 +17,13 @@
 //               K=32) four times per 128-K block, selecting the UE8M0 byte of
 //               the current K-block with the scale-factor id, and commits
 //               stage releases and accumulator hand-offs to mbarriers.
-//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld), fp32 -> bf16 with
-//               round-to-nearest-even, predicated row stores. Rows past the
-//               valid count (masked_m, padding of m_indices, M) are never
-//               written.
+//   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld, up to 128 columns
+//               per batch; TMEM is handed back right after the last read),
+//               fp32 -> bf16 with round-to-nearest-even, 32x32 chunks staged
+//               in swizzled shared memory and written by TMA; chunks holding
+//               rows that must not be written (past masked_m, padding of
+//               m_indices) use predicated row stores instead, so those rows
+//               are never touched.
 // The accumulator is double-buffered in TMEM when two fit next to the scale
 // columns, so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
@@ -58,6 +61,7 @@ constexpr uint32_t DEVERR_MIXED_EXPERT_BLOCK = 2u;
 struct GemmParams {
     CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous) or 3-D {K, max_m, G} (masked)
     CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped)
+    CUtensorMap tma_d;        // D (bf16, store): 2-D {N, rows} or 3-D {N, max_m, G}; 32x32 box, 64-byte swizzle
     const int32_t* sfa;       // packed scale rows of A
     const int32_t* sfb;       // packed scale rows of B (per 128 rows, per group)
     __nv_bfloat16* d;         // output
@@ -77,14 +81,17 @@ struct GemmParams {
 
 template <int BN>
 struct GemmConfig {
-    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "N tile must be a multiple of 16 in [16, 256]");
+    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 32 in [32, 256]");
     static constexpr int A_BYTES = BM * BK;
     static constexpr int B_BYTES = BN * BK;
     static constexpr int SFB_CHUNKS = (BN + 127) / 128;         // 128-column chunks of B scales
     static constexpr int SFA_BYTES = 512;                       // 32 rows x 16 bytes
     static constexpr int SFB_BYTES = 512 * SFB_CHUNKS;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int FIXED_BYTES = 1024 /*align slack*/ + 512 /*barriers*/ + (2 * MAX_MASKED_GROUPS + 8) * 4;
+    static constexpr int EPI_WARP_BYTES = 2 * 2048;                // two 32x32 bf16 staging buffers per warp
+    static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
+    static constexpr int FIXED_BYTES =
+        1024 /*align slack*/ + EPI_BYTES + 512 /*barriers*/ + (2 * MAX_MASKED_GROUPS + 8) * 4;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static_assert(STAGES >= 2, "pipeline too shallow");
@@ -254,7 +261,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* smem_a = smem;                                         // STAGES x 16 KB
     uint8_t* smem_b = smem_a + STAGES * Cfg::A_BYTES;               // STAGES x BN*128
-    uint8_t* smem_sfa = smem_b + STAGES * Cfg::B_BYTES;             // STAGES x 512
+    uint8_t* smem_epi = smem_b + STAGES * Cfg::B_BYTES;             // 4 warps x 2 x 2 KB (1024-aligned)
+    uint8_t* smem_sfa = smem_epi + Cfg::EPI_BYTES;                  // STAGES x 512
     uint8_t* smem_sfb = smem_sfa + STAGES * Cfg::SFA_BYTES;         // STAGES x 512*chunks
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem_sfb + STAGES * Cfg::SFB_BYTES);
     uint64_t* full_bar = bars;                    // TMA bytes + scale words landed
@@ -286,6 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.tma_a);
         tma_prefetch_desc(&p.tma_b);
+        tma_prefetch_desc(&p.tma_d);
     }
     if (warp == 1) {
         tmem_alloc(s_tmem, Cfg::TMEM_COLS);
@@ -458,10 +467,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         wait_quiet(drain_bar, 0, p.wait_limit_ns);
     } else {
         // ------------------------------------------------------- epilogue --
+        // Each warp owns 32 rows (its TMEM sub-partition). Per tile it reads
+        // the accumulator in batches of up to 128 columns, hands TMEM back to
+        // the MMA warp right after the last read, and then writes bf16:
+        // 32x32 chunks staged in swizzled shared memory and stored with TMA
+        // when all 32 rows may be written, predicated 16-byte stores otherwise.
         const int q = static_cast<int>(warp & 3);   // TMEM sub-partition of this warp
+        uint8_t* stg = smem_epi + (warp - 2) * Cfg::EPI_WARP_BYTES;
         int acc = 0;
         uint32_t acc_phase = 0;
         int gcur = 0;
+        int buf = 0;
         Tile c;
         for (int t = blockIdx.x; next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, c, lane); t += gridDim.x) {
             const int mloc = c.m_blk * BM + 32 * q + static_cast<int>(lane);
@@ -480,44 +496,76 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 if (in_range && id != c.g) atomicOr(p.status, DEVERR_MIXED_EXPERT_BLOCK);
                 out_row = static_cast<size_t>(mloc);
             }
+            // TMA stores clip at the tensor's edges, so for the dense form rows
+            // past M are safe; the grouped forms need every row of the chunk valid.
+            const bool use_tma = (KIND == kDense) ? true : (__all_sync(0xffffffffu, valid) != 0);
+            const int row_coord = c.m_blk * BM + 32 * q;
             if (!wait_bounded(&tfull_bar[acc], acc_phase, p, s_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_COLS;
             const int n0 = c.n_blk * BN;
             __nv_bfloat16* drow = p.d + out_row * static_cast<size_t>(p.n) + n0;
-#pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
-                uint32_t r[32];
-                constexpr int TAIL = BN % 32;
-                const bool full32 = (TAIL == 0) || (c0 + 32 <= BN);
-                if (full32) tmem_ld_32x32b_x32(taddr + c0, r);
-                else tmem_ld_32x32b_x16(taddr + c0, r);
+#pragma unroll
+            for (int h = 0; h < BN; h += 128) {
+                constexpr int kMaxBatch = 128;
+                const int cols = (BN - h) < kMaxBatch ? (BN - h) : kMaxBatch;  // compile-time after unrolling
+                uint32_t r[kMaxBatch];
+#pragma unroll
+                for (int j = 0; j < kMaxBatch / 32; ++j)
+                    if (32 * j < cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
                 tc_wait_ld();
-                if (c0 + 32 >= BN) {
+                if (h + 128 >= BN) {
                     // last TMEM read of this accumulator: hand it back to the MMA warp
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty_bar[acc]);
                 }
-                if (valid) {
-                    const int nv = full32 ? 4 : 2;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (v < nv && n0 + c0 + 8 * v < p.n) {
-                            uint32_t w[4];
+                for (int j = 0; j < kMaxBatch / 32; ++j) {
+                    if (32 * j >= cols) continue;
+                    const int col = n0 + h + 32 * j;
+                    if (col >= p.n) continue;  // warp-uniform: N tail
+                    uint32_t w[16];
 #pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[8 * v + 2 * h]),
-                                                                          __uint_as_float(r[8 * v + 2 * h + 1]));
-                                w[h] = *reinterpret_cast<uint32_t*>(&b2);
-                            }
-                            *reinterpret_cast<uint4*>(drow + c0 + 8 * v) = make_uint4(w[0], w[1], w[2], w[3]);
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[32 * j + 2 * i]),
+                                                                  __uint_as_float(r[32 * j + 2 * i + 1]));
+                        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+                    }
+                    if (use_tma) {
+                        // the store issued two chunks ago has finished reading this buffer
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        uint8_t* sb = stg + buf * 2048;
+                        // 32 rows x 64 bytes with the 64-byte swizzle: granule g of
+                        // row r sits at granule g ^ ((r >> 1) & 3)
+                        const uint32_t sw = (lane >> 1) & 3u;
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
+                                make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
+                            else tma_store_2d(&p.tma_d, sb, col, row_coord);
+                            bulk_commit_group();
                         }
+                        buf ^= 1;
+                    } else if (valid) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            if (col + 8 * v < p.n)
+                                *reinterpret_cast<uint4*>(drow + h + 32 * j + 8 * v) =
+                                    make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
                     }
                 }
             }
             if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
         }
+        // every bulk store must have completed before the CTA exits
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     tc_fence_before();

@@ -15,7 +15,7 @@ from helpers import bf16_to_f64, check_fp, fill_sentinel, is_sentinel
 
 pytestmark = pytest.mark.gpu
 
-BLOCK_NS = [64, 128, 176, 224, 256]
+BLOCK_NS = [64, 96, 128, 160, 192, 224, 256]
 
 
 @pytest.fixture(autouse=True)
@@ -135,7 +135,7 @@ def check_masked(p, d, masked_m=None, what="masked"):
     check_fp(bf16_to_f64(d)[valid], ref[valid], what)
 
 
-@pytest.mark.parametrize("bn", [64, 128, 176, 256])
+@pytest.mark.parametrize("bn", [64, 96, 160, 256])
 def test_masked_parity_and_sentinel(bn):
     mm = np.array([0, 1, 128, 200, 77, -3, 500], dtype=np.int32)
     p = W.masked(mm, 200, 272, 384, seed=11)
@@ -195,7 +195,7 @@ def check_contig(p, d, m_indices=None, what="contiguous"):
     check_fp(bf16_to_f64(d)[valid], ref[valid], what)
 
 
-@pytest.mark.parametrize("bn", [64, 128, 224, 256])
+@pytest.mark.parametrize("bn", [64, 192, 224, 256])
 def test_contiguous_parity_and_padding(bn):
     p = W.contiguous([5, 0, 130, 128, 1], 264, 512, seed=21, tail_blocks=1)
     d = run_contig(p, bn=bn)
