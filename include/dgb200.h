@@ -105,6 +105,16 @@ DG_API dg_status dgb200_set_block_n(int block_n);
 DG_API int dgb200_block_n_supported(int block_n);
 
 /*
+ * Force the dense GEMM to run on single CTAs (1) or on CTA pairs (2, tcgen05
+ * cta_group::2 with a 256-row tile); 0 restores the heuristic. The grouped
+ * forms always use single CTAs. Process-wide; meant for tests and tuning.
+ * Returns DG_ERR_UNSUPPORTED for other values; a forced combination of tile
+ * width and group that is not built makes the GEMM calls return
+ * DG_ERR_UNSUPPORTED.
+ */
+DG_API dg_status dgb200_set_cta_group(int cta_group);
+
+/*
  * Test hook for the failure path (process-wide). wait_limit_ms bounds every
  * wait inside the GEMM kernels (0 restores the default, 2000 ms). mode 1 makes
  * CTA 0 of each GEMM launch withhold the arrive of its first pipeline stage,

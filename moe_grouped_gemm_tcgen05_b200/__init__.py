@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-    "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks",
+    "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -76,6 +76,8 @@ def load():
         L.dgb200_set_block_n.argtypes = [i32]
         L.dgb200_block_n_supported.restype = i32
         L.dgb200_block_n_supported.argtypes = [i32]
+        L.dgb200_set_cta_group.restype = i32
+        L.dgb200_set_cta_group.argtypes = [i32]
         L.dgb200_set_test_hooks.restype = i32
         L.dgb200_set_test_hooks.argtypes = [i32, i32]
         L.fp8_gemm_nt.restype = i32
@@ -138,6 +140,11 @@ def device_error(clear: bool = True) -> int:
 def set_block_n(block_n: int):
     """Force the N tile width (0 = heuristic). For tests and tuning."""
     _check("dgb200_set_block_n", load().dgb200_set_block_n(int(block_n)))
+
+
+def set_cta_group(cta_group: int):
+    """Force single CTAs (1) or CTA pairs (2) for the dense GEMM (0 = heuristic)."""
+    _check("dgb200_set_cta_group", load().dgb200_set_cta_group(int(cta_group)))
 
 
 def set_test_hooks(mode: int = 0, wait_limit_ms: int = 0):

@@ -11,6 +11,7 @@
 
 #include <atomic>
 #include <cstdint>
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -32,43 +33,54 @@ struct DeviceState {
     bool ready = false;
     int sms = 0;
     uint32_t* status = nullptr;  // address of g_dg_device_status on this device
+    int max_pairs[64] = {};      // co-resident CTA pairs per kernel entry (cluster kernels only)
 };
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_bn{0};
+std::atomic<int> g_force_cg{0};
 std::atomic<int> g_test_mode{0};
 std::atomic<uint64_t> g_wait_limit_ns{dg::DEFAULT_WAIT_LIMIT_NS};
+// DGB200_LOG=1 in the environment prints each GEMM launch's configuration to stderr.
+const bool g_log = [] {
+    const char* v = std::getenv("DGB200_LOG");
+    return v != nullptr && v[0] == '1';
+}();
+// DGB200_K_ROTATE=1 makes every tile start its K walk at a rotated group (default: in order).
+const int g_k_rotate = [] {
+    const char* v = std::getenv("DGB200_K_ROTATE");
+    return (v != nullptr && v[0] == '1') ? 1 : 0;
+}();
 
 // --------------------------------------------------------------- kernels ----
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG>
 void* kernel_ptr() {
-    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND>);
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG>);
 }
 
 struct KernelEntry {
     int bn;
     int kind;
+    int cg;     // CTAs per MMA unit (1, or a cluster pair)
     void* fn;
     int smem;
 };
 
-#define DG_ENTRY(BN, KIND) {BN, KIND, kernel_ptr<BN, KIND>(), dg::GemmConfig<BN>::SMEM_BYTES}
-#define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense), DG_ENTRY(BN, dg::kContiguous), DG_ENTRY(BN, dg::kMasked)
+#define DG_ENTRY(BN, KIND, CG) \
+    {BN, KIND, CG, kernel_ptr<BN, KIND, CG>(), dg::GemmConfig<BN, CG, KIND == dg::kMasked>::SMEM_BYTES}
+#define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1)
 
 const KernelEntry kKernels[] = {
     DG_ALL_KINDS(64),  DG_ALL_KINDS(96),  DG_ALL_KINDS(128), DG_ALL_KINDS(160),
     DG_ALL_KINDS(192), DG_ALL_KINDS(224), DG_ALL_KINDS(256),
+    DG_ENTRY(128, dg::kDense, 2), DG_ENTRY(160, dg::kDense, 2), DG_ENTRY(192, dg::kDense, 2),
+    DG_ENTRY(224, dg::kDense, 2), DG_ENTRY(256, dg::kDense, 2),
 };
+constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
-
-const KernelEntry* find_kernel(int bn, int kind) {
-    for (const auto& e : kKernels)
-        if (e.bn == bn && e.kind == kind) return &e;
-    return nullptr;
-}
 
 // ------------------------------------------------------------------ init ----
 
@@ -91,9 +103,28 @@ dg_status init_device(int dev) {
         return DG_ERR_CUDA;
     if (major != 10 || minor != 0) return DG_ERR_UNSUPPORTED;  // built for sm_100a only
     if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
-    for (const auto& e : kKernels) {
+    static_assert(kNumKernels <= 64, "DeviceState::max_pairs too small");
+    for (int i = 0; i < kNumKernels; ++i) {
+        const KernelEntry& e = kKernels[i];
         if (cudaFuncSetAttribute(e.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, e.smem) != cudaSuccess)
             return DG_ERR_CUDA;
+        if (e.cg == 2) {
+            // how many CTA pairs fit on the device at once (pairs must share a GPC)
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(2 * (st.sms / 2));
+            cfg.blockDim = dim3(dg::NUM_THREADS);
+            cfg.dynamicSmemBytes = static_cast<size_t>(e.smem);
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, e.fn, &cfg) != cudaSuccess || clusters < 1) return DG_ERR_CUDA;
+            st.max_pairs[i] = clusters;
+        }
     }
     void* status = nullptr;
     if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
@@ -149,34 +180,53 @@ constexpr double kL2BytesPerClk = 64.0;
 // (the MMA warp waits for the epilogue's TMEM reads).
 constexpr double kSingleBufferBubble = 600.0;
 
-// Clocks one CTA spends per 128-K block of a (rows_a x bn) tile: the larger of
-// the tensor core (four K=32 MMAs of bn/2 clocks), shared-memory reads
-// (4 x (4 KB of A + 32*bn of B) at 128 B/clk) and the L2 feed of the stage.
-double kblock_clocks(int bn, int rows_a) {
+// Clocks one SM spends per 128-K block of its (rows_a x bn) share of a tile:
+// the larger of the tensor core (four K=32 MMAs of bn/2 clocks), shared-memory
+// reads (4 x (4 KB of A + 32*bn/cg of B) at 128 B/clk) and the L2 feed of the
+// stage (rows_a + bn/cg rows of 128 bytes).
+double kblock_clocks(int bn, int cg, int rows_a) {
     const double tc = 2.0 * bn;
-    const double sm = 4.0 * (4096.0 + 32.0 * bn) / 128.0;
-    const double l2 = (rows_a + bn) * 128.0 / kL2BytesPerClk;
+    const double sm = 4.0 * (4096.0 + 32.0 * bn / cg) / 128.0;
+    const double l2 = (rows_a + static_cast<double>(bn) / cg) * 128.0 / kL2BytesPerClk;
     double t = tc > sm ? tc : sm;
     return t > l2 ? t : l2;
 }
 
-int num_acc_for(int bn) { return (2 * bn + 4 + 4 * ((bn + 127) / 128) <= 512) ? 2 : 1; }
+int num_acc_for(int bn) { return (2 * bn + 2 * (4 + 4 * ((bn + 127) / 128)) <= 512) ? 2 : 1; }
 
-// Pick the N tile with the least modelled time: waves of tiles x time per tile.
-int choose_block_n(long long m_blocks, int rows_a, int n, int kb, int sms) {
-    const int forced = g_force_bn.load();
-    if (forced != 0) return forced;
-    int best = 128;
+struct TileChoice {
+    const KernelEntry* entry;
+    int units;  // concurrent MMA units (CTAs, or CTA pairs)
+};
+
+// Pick the kernel (N tile, one CTA or a CTA pair) with the least modelled
+// time: waves of tiles over the concurrent MMA units x time per tile.
+TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int kb, long long m128_blocks) {
+    const int forced_bn = g_force_bn.load();
+    const int forced_cg = kind == dg::kDense ? g_force_cg.load() : 0;  // pairs exist for the dense form only
+    TileChoice best{nullptr, 0};
     double best_cost = 1e300;
-    for (int bn : kBlockNs) {
-        const long long nb = (n + bn - 1) / bn;
-        const long long tiles = m_blocks * nb;
-        const long long waves = (tiles + sms - 1) / sms;
-        const double tile = kb * kblock_clocks(bn, rows_a) + (num_acc_for(bn) == 1 ? kSingleBufferBubble : 0.0);
+    for (int i = 0; i < kNumKernels; ++i) {
+        const KernelEntry& e = kKernels[i];
+        if (e.kind != kind) continue;
+        if (forced_bn != 0 && e.bn != forced_bn) continue;
+        if (forced_cg != 0 && e.cg != forced_cg) continue;
+        if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
+        const int units = e.cg == 1 ? st->sms : st->max_pairs[i];
+        if (units < 1) continue;
+        const long long mt = (m128_blocks + e.cg - 1) / e.cg;
+        const long long nb = (n + e.bn - 1) / e.bn;
+        const long long waves = (mt * nb + units - 1) / units;
+        const int rows_a = rows < dg::BM ? rows : dg::BM;
+        const double tile =
+            kb * kblock_clocks(e.bn, e.cg, rows_a) + (num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0);
         const double cost = static_cast<double>(waves) * tile;
-        if (cost < best_cost * 0.999 || (cost <= best_cost * 1.001 && bn > best)) {
+        const bool better = cost < best_cost * 0.999 ||
+                            (cost <= best_cost * 1.001 && best.entry && (e.cg > best.entry->cg ||
+                                                                         (e.cg == best.entry->cg && e.bn > best.entry->bn)));
+        if (best.entry == nullptr || better) {
             best_cost = cost;
-            best = bn;
+            best = TileChoice{&e, units};
         }
     }
     return best;
@@ -198,28 +248,46 @@ dg_status check_common(const void* a, const int32_t* sfa, const void* b, const i
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
                       void* stream, DeviceState* st, const void* a, const void* b, int a_rank, int b_rank,
                       uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
-    const int rows_a = p.rows < dg::BM ? p.rows : dg::BM;
-    const int bn = choose_block_n(m_blocks_for_heuristic, rows_a, p.n, p.k / 128, st->sms);
-    const KernelEntry* e = find_kernel(bn, kind);
+    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k / 128, m_blocks_for_heuristic);
+    const KernelEntry* e = choice.entry;
     if (e == nullptr) return DG_ERR_UNSUPPORTED;
+    const int bn = e->bn;
+    const int cg = e->cg;
     p.status = st->status;
     p.kb = p.k / 128;
     p.kp = (p.kb + 3) / 4;
     p.nb_sf = (p.n + 127) / 128;
     p.num_n_blocks = (p.n + bn - 1) / bn;
-    p.raster_group = 16;
+    if (cg == 2) p.num_m_blocks = (p.rows + 2 * dg::BM - 1) / (2 * dg::BM);
+    p.raster_group = 16 / cg;
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.test_mode = g_test_mode.load();
+    p.k_rotate = g_k_rotate;
     if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
-    if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn)))
+    if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats,
+                          static_cast<uint32_t>(bn / cg)))
         return DG_ERR_INVALID_ARG;
     if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
-    const long long tiles = max_tiles_per_nblock * p.num_n_blocks;
+    const long long tiles = (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks);
     if (tiles <= 0) return DG_OK;
-    const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+    const int units = static_cast<int>(tiles < choice.units ? tiles : choice.units);
     void* args[] = {&p};
-    cudaError_t err = cudaLaunchKernel(e->fn, dim3(grid), dim3(dg::NUM_THREADS), args, static_cast<size_t>(e->smem),
-                                       static_cast<cudaStream_t>(stream));
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cg);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(static_cast<unsigned>(units * cg));
+    cfg.blockDim = dim3(dg::NUM_THREADS);
+    cfg.dynamicSmemBytes = static_cast<size_t>(e->smem);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = attr;
+    cfg.numAttrs = cg == 2 ? 1 : 0;
+    if (g_log)
+        std::fprintf(stderr, "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d grid=%d (units %d) smem=%d\n",
+                     kind, p.rows, p.n, p.k, p.groups, bn, cg, units * cg, choice.units, e->smem);
+    cudaError_t err = cudaLaunchKernelExC(&cfg, e->fn, args);
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
@@ -264,6 +332,12 @@ int dgb200_block_n_supported(int block_n) {
 dg_status dgb200_set_block_n(int block_n) {
     if (block_n != 0 && !dgb200_block_n_supported(block_n)) return DG_ERR_UNSUPPORTED;
     g_force_bn.store(block_n);
+    return DG_OK;
+}
+
+dg_status dgb200_set_cta_group(int cta_group) {
+    if (cta_group < 0 || cta_group > 2) return DG_ERR_UNSUPPORTED;
+    g_force_cg.store(cta_group);
     return DG_OK;
 }
 

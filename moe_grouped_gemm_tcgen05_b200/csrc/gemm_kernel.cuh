@@ -7,16 +7,19 @@
 // Grouped GEMMs" for the masked form; the contiguous form is the "continuous
 // storage layout" of "DeepGEMM tested by Novita AI").
 //
-// CTA = 6 warps, one CTA per SM, grid fixed by the problem sizes:
-//   warp 0      producer: TMA loads of the A and B tiles (128-byte swizzle)
-//               into a STAGES-deep shared-memory ring; every 4th K-block it
-//               also gathers the packed scale words (one int32 = 4 K-blocks)
-//               into the 32x16-byte layout that tcgen05.cp expects.
-//   warp 1      MMA issuer: allocates TMEM, copies the scale words to TMEM,
-//               issues tcgen05.mma.kind::mxf8f6f4.block_scale (M=128, N=BN,
-//               K=32) four times per 128-K block, selecting the UE8M0 byte of
-//               the current K-block with the scale-factor id, and commits
-//               stage releases and accumulator hand-offs to mbarriers.
+// CTA = 7 warps, one CTA per SM, persistent over a grid fixed by the sizes:
+//   warp 0      TMA producer: loads of the A and B tiles (128-byte swizzle)
+//               into a STAGES-deep shared-memory ring.
+//   warp 6      scale producer: per group of four K-blocks (one packed int32
+//               per row/column) gathers the scale words into the 32x16-byte
+//               layout that tcgen05.cp expects, into its own 4-deep ring,
+//               loads issued one group ahead.
+//   warp 1      MMA issuer: allocates TMEM, copies each group's scale words to
+//               TMEM (and frees their slot as soon as the copy completes),
+//               issues tcgen05.mma.kind::mxf8f6f4.block_scale (K=32) four
+//               times per 128-K block, selecting the UE8M0 byte of the
+//               current K-block with the scale-factor id, and commits stage
+//               releases and accumulator hand-offs to mbarriers.
 //   warps 2..5  epilogue: TMEM -> registers (tcgen05.ld, up to 128 columns
 //               per batch; TMEM is handed back right after the last read),
 //               fp32 -> bf16 with round-to-nearest-even, 32x32 chunks staged
@@ -26,6 +29,17 @@
 //               are never touched.
 // The accumulator is double-buffered in TMEM when two fit next to the scale
 // columns, so the epilogue of tile i overlaps the MMAs of tile i+1.
+//
+// CG = 2 runs a cluster of two CTAs as one MMA unit (tcgen05 cta_group::2):
+// a 256 x BN tile whose A rows are split 128/128 and whose B rows are split
+// BN/2 / BN/2 between the two CTAs' shared memory. Only the even CTA (the
+// leader) issues MMAs and tcgen05 copies (all with cta_group::2); both CTAs'
+// TMA loads complete on the leader's stage barrier, the odd CTA publishes its
+// scale words with a cluster-scope release on the leader's scale barrier
+// (the scale ring gives that release several groups of slack), and commits
+// reach both CTAs' barriers. Each CTA's TMEM holds its 128 rows x BN of the
+// accumulator, its own A scales and the full-width B scales. Per SM this
+// halves the B bytes each 128-K block needs. No load is multicast.
 //
 // Block scaling: the hardware MMA applies one UE8M0 scale per 32 K values for
 // each row of A and each column of B. The 128-granular scales of this format
@@ -38,6 +52,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda.h>
 
@@ -47,10 +62,11 @@ namespace dg {
 
 enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
-constexpr int BM = 128;                 // rows per tile (one MMA, cta_group::1)
+constexpr int BM = 128;                 // rows of A per CTA
 constexpr int BK = 128;                 // K per pipeline stage = one scale block
 constexpr int MMA_K = 32;               // K of one kind::mxf8f6f4 MMA
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 224;
+constexpr int SF_RING = 4;              // scale-word groups in flight
 constexpr int MAX_MASKED_GROUPS = 1024;
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
 constexpr uint64_t DEFAULT_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
@@ -60,7 +76,7 @@ constexpr uint32_t DEVERR_MIXED_EXPERT_BLOCK = 2u;
 
 struct GemmParams {
     CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous) or 3-D {K, max_m, G} (masked)
-    CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped)
+    CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped); box BN/CG rows
     CUtensorMap tma_d;        // D (bf16, store): 2-D {N, rows} or 3-D {N, max_m, G}; 32x32 box, 64-byte swizzle
     const int32_t* sfa;       // packed scale rows of A
     const int32_t* sfb;       // packed scale rows of B (per 128 rows, per group)
@@ -72,40 +88,48 @@ struct GemmParams {
     int kb;                   // K / 128
     int kp;                   // ceil(kb / 4) packed words per scale row
     int nb_sf;                // ceil(N / 128) scale rows per weight matrix
-    int num_m_blocks;         // ceil(rows / 128)
+    int num_m_blocks;         // ceil(rows / (128 * CG)) m-tiles
     int num_n_blocks;         // ceil(N / BN)
-    int raster_group;         // m-blocks per raster band (dense / contiguous)
+    int raster_group;         // m-tiles per raster band (dense / contiguous)
     uint64_t wait_limit_ns;   // bound of every mbarrier wait
+    int k_rotate;             // 1: each tile walks its K groups starting at group (tile mod groups)
     int test_mode;            // 1: CTA 0 withholds one stage arrive (exercises the timeout path)
 };
 
-template <int BN>
+template <int BN, int CG, bool SCHED_SMEM>
 struct GemmConfig {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 32 in [32, 256]");
+    static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
+    static constexpr int B_ROWS = BN / CG;                      // rows of B in this CTA's shared memory
     static constexpr int A_BYTES = BM * BK;
-    static constexpr int B_BYTES = BN * BK;
-    static constexpr int SFB_CHUNKS = (BN + 127) / 128;         // 128-column chunks of B scales
+    static constexpr int B_BYTES = B_ROWS * BK;
+    static constexpr int SFB_CHUNKS = (BN + 127) / 128;         // 128-column chunks of B scales (full width)
     static constexpr int SFA_BYTES = 512;                       // 32 rows x 16 bytes
     static constexpr int SFB_BYTES = 512 * SFB_CHUNKS;
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    static constexpr int EPI_WARP_BYTES = 2 * 2048;                // two 32x32 bf16 staging buffers per warp
+    static constexpr int SF_SLOT_BYTES = SFA_BYTES + SFB_BYTES;  // one group of scale words
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr uint32_t TX_BYTES = CG * (A_BYTES + B_BYTES);  // TMA bytes per stage, both CTAs
+    static constexpr int EPI_WARP_BYTES = 2 * 2048;             // two 32x32 bf16 staging buffers per warp
     static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
+    static constexpr int SCHED_BYTES = SCHED_SMEM ? (2 * MAX_MASKED_GROUPS + 8) * 4 : 64;
     static constexpr int FIXED_BYTES =
-        1024 /*align slack*/ + EPI_BYTES + 512 /*barriers*/ + (2 * MAX_MASKED_GROUPS + 8) * 4;
+        1024 /*align slack*/ + EPI_BYTES + SF_RING * SF_SLOT_BYTES + 512 /*barriers*/ + SCHED_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
     static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
     static_assert(STAGES >= 2, "pipeline too shallow");
     static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES;
 
-    // TMEM columns: accumulator slot(s), then 4 columns of A scales and
-    // 4 per 128-column chunk of B scales.
-    static constexpr int ACC_COLS = ((BN + 31) / 32) * 32;
+    // TMEM columns: accumulator slot(s) of BN columns, then two sets of scale
+    // columns (4 of A scales and 4 per 128-column chunk of B scales), used by
+    // alternate groups so that the copy of the next group's scales never
+    // overwrites words that MMAs still in the pipe are reading.
+    static constexpr int ACC_COLS = BN;
     static constexpr int SF_COLS = 4 + 4 * SFB_CHUNKS;
-    static constexpr int NUM_ACC = (2 * ACC_COLS + SF_COLS <= 512) ? 2 : 1;
-    static constexpr int SFA_COL = NUM_ACC * ACC_COLS;
-    static constexpr int SFB_COL = SFA_COL + 4;
-    static_assert(SFB_COL + 4 * SFB_CHUNKS <= 512, "TMEM overflow");
+    static constexpr int NUM_ACC = (2 * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1;
+    static constexpr int SF_BASE = NUM_ACC * ACC_COLS;
+    static_assert(SF_BASE + 2 * SF_COLS <= 512, "TMEM overflow");
     static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t IDESC = idesc_mxf8_e4m3_ue8m0(BM * CG, BN);
 };
 
 struct Tile {
@@ -123,16 +147,42 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Wait for the phase of `bar` with the given parity. Gives up when another
 // role of this CTA has given up, or after p.wait_limit_ns; a timeout is
 // recorded in the device status word.
+// CLUSTER_ACQUIRE: the phase publishes shared-memory data written by the peer
+// CTA of a pair (its scale words), so the probe acquires at cluster scope.
+template <bool CLUSTER_ACQUIRE = false>
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const GemmParams& p,
                                              volatile int* s_abort) {
-    if (mbar_try_wait(bar, parity)) return true;
+    auto probe = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (probe()) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (probe()) return true;
         if (*s_abort) return false;
         if (global_ns() - t0 > p.wait_limit_ns) {
             atomicOr(p.status, DEVERR_TIMEOUT);
             *s_abort = 1;
+            return false;
+        }
+    }
+}
+
+// Warp-wide form of wait_bounded: every lane probes and the outcome is a vote,
+// so all 32 lanes leave together with the same answer. Roles that issue
+// tcgen05 instructions under elect.sync use it: a lane that left a loop early
+// would leave the others waiting at the next elect.sync.
+template <bool CLUSTER_ACQUIRE = false>
+__device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const GemmParams& p, volatile int* s_abort) {
+    auto probe = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    if (__all_sync(0xffffffffu, probe())) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        if (__all_sync(0xffffffffu, probe())) return true;
+        const bool late = global_ns() - t0 > p.wait_limit_ns;
+        if (__any_sync(0xffffffffu, late || *s_abort != 0)) {
+            if (__any_sync(0xffffffffu, late) && lane_id() == 0) {
+                atomicOr(p.status, DEVERR_TIMEOUT);
+                *s_abort = 1;
+            }
             return false;
         }
     }
@@ -145,10 +195,16 @@ __device__ __forceinline__ void wait_quiet(uint64_t* bar, uint32_t parity, uint6
     }
 }
 
+__device__ __forceinline__ void sleep_ns(uint64_t ns) {
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < ns) {
+    }
+}
+
 // ------------------------------------------------------------- scheduling --
 
-// Dense / contiguous: banded raster. Within a band of `raster_group` m-blocks
-// the m-block varies fastest, so CTAs running at the same time share the B tile
+// Dense / contiguous: banded raster. Within a band of `raster_group` m-tiles
+// the m-tile varies fastest, so CTAs running at the same time share the B tile
 // and a bounded slab of A.
 __device__ __forceinline__ bool raster_tile(const GemmParams& p, int t, Tile& c) {
     const int total = p.num_m_blocks * p.num_n_blocks;
@@ -205,36 +261,44 @@ __device__ __forceinline__ bool next_tile(const GemmParams& p, const int* s_pref
     }
 }
 
+// Group of four K-blocks visited at step gi of tile t. Rotating the start by
+// the tile index makes CTAs that share an A or B tile (and run in lockstep)
+// touch its K-blocks at different times, so only one of them waits for DRAM
+// per block and the others are served from L2. Whole groups keep the packed
+// scale words aligned; only the order of the fp32 accumulation changes.
+__device__ __forceinline__ int rot_group(const GemmParams& p, int t, int gi, int kg_count) {
+    return p.k_rotate ? (gi + t) % kg_count : gi;
+}
+
 // ------------------------------------------------------- scale-word gather --
 
-// Scale words of one 4-K-block group for a tile: lane r holds, for j = 0..3,
-// the word of A row 32j + r and, per 128-column chunk, the word of B column
-// 128*chunk + 32j + r. Stored as one 16-byte row per lane, this is the
-// 32x128-bit matrix whose copy to TMEM puts row m at lane m % 32, column m / 32.
+// Scale words of one 4-K-block group for this CTA's part of a tile: lane r
+// holds, for j = 0..3, the word of A row row0 + 32j + r and, per 128-column
+// chunk, the word of B column n0 + 128*chunk + 32j + r. Stored as one 16-byte
+// row per lane, this is the 32x128-bit matrix whose copy to TMEM puts row m at
+// lane m % 32, column m / 32.
 template <int BN, int KIND>
 struct ScaleWords {
-    static constexpr int CH = GemmConfig<BN>::SFB_CHUNKS;
+    static constexpr int CH = (BN + 127) / 128;
     uint32_t a[4];
     uint32_t b[CH][4];
 
-    __device__ __forceinline__ void load(const GemmParams& p, const Tile& c, int kg, uint32_t lane) {
+    __device__ __forceinline__ void load(const GemmParams& p, int row0, int n0, int g, int kg, uint32_t lane) {
         // A rows: clamp into the operand so every load is in bounds; rows past
         // the valid count only feed accumulator rows that are never stored.
         size_t row_base = 0;
-        int row_lim = p.rows;
-        if constexpr (KIND == kMasked) row_base = static_cast<size_t>(c.g) * p.rows;
+        if constexpr (KIND == kMasked) row_base = static_cast<size_t>(g) * p.rows;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int r = min(c.m_blk * BM + 32 * j + static_cast<int>(lane), row_lim - 1);
+            const int r = min(row0 + 32 * j + static_cast<int>(lane), p.rows - 1);
             a[j] = static_cast<uint32_t>(__ldg(p.sfa + (row_base + r) * p.kp + kg));
         }
-        const int g = (KIND == kDense) ? 0 : max(c.g, 0);
-        const int32_t* sfb = p.sfb + static_cast<size_t>(g) * p.nb_sf * p.kp;
+        const int32_t* sfb = p.sfb + static_cast<size_t>(KIND == kDense ? 0 : max(g, 0)) * p.nb_sf * p.kp;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int col = c.n_blk * BN + 128 * ch + 32 * j + static_cast<int>(lane);
+                const int col = n0 + 128 * ch + 32 * j + static_cast<int>(lane);
                 const int nb = min(col / 128, p.nb_sf - 1);
                 b[ch][j] = static_cast<uint32_t>(__ldg(sfb + static_cast<size_t>(nb) * p.kp + kg));
             }
@@ -251,41 +315,51 @@ struct ScaleWords {
 
 // ------------------------------------------------------------------ kernel --
 
-template <int BN, int KIND>
+template <int BN, int KIND, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
-    using Cfg = GemmConfig<BN>;
+    static_assert(CG == 1 || KIND == kDense, "CTA pairs are built for the dense form");
+    using Cfg = GemmConfig<BN, CG, KIND == kMasked>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int NUM_ACC = Cfg::NUM_ACC;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* smem_a = smem;                                         // STAGES x 16 KB
-    uint8_t* smem_b = smem_a + STAGES * Cfg::A_BYTES;               // STAGES x BN*128
+    uint8_t* smem_b = smem_a + STAGES * Cfg::A_BYTES;               // STAGES x B_ROWS*128
     uint8_t* smem_epi = smem_b + STAGES * Cfg::B_BYTES;             // 4 warps x 2 x 2 KB (1024-aligned)
-    uint8_t* smem_sfa = smem_epi + Cfg::EPI_BYTES;                  // STAGES x 512
-    uint8_t* smem_sfb = smem_sfa + STAGES * Cfg::SFA_BYTES;         // STAGES x 512*chunks
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_sfb + STAGES * Cfg::SFB_BYTES);
-    uint64_t* full_bar = bars;                    // TMA bytes + scale words landed
+    uint8_t* smem_sf = smem_epi + Cfg::EPI_BYTES;                   // SF_RING x (A scales, B scales)
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem_sf + SF_RING * Cfg::SF_SLOT_BYTES);
+    uint64_t* full_bar = bars;                    // A/B bytes landed (the leader's counts both CTAs)
     uint64_t* empty_bar = bars + STAGES;          // MMAs reading the stage finished
-    uint64_t* tfull_bar = bars + 2 * STAGES;      // accumulator ready for the epilogue
-    uint64_t* tempty_bar = tfull_bar + 2;         // accumulator drained by the epilogue
-    uint64_t* drain_bar = tempty_bar + 2;         // all MMAs of this CTA finished
+    uint64_t* sf_full_bar = bars + 2 * STAGES;    // scale words of a group stored (every CTA of the unit)
+    uint64_t* sf_empty_bar = sf_full_bar + SF_RING;  // scale words copied into TMEM
+    uint64_t* tfull_bar = sf_empty_bar + SF_RING;    // accumulator ready for the epilogue
+    uint64_t* tempty_bar = tfull_bar + 2;            // accumulator drained by the epilogue(s)
+    uint64_t* drain_bar = tempty_bar + 2;            // all MMAs issued for this CTA finished
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
-    int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1]
-    int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups]
+    int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked)
+    int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups]     (masked)
 
     const uint32_t warp = threadIdx.x / 32;
     const uint32_t lane = lane_id();
+    const uint32_t rank = (CG == 1) ? 0u : cluster_ctarank();    // position in the CTA pair
+    const bool leader = rank == 0;
+    const int unit = static_cast<int>(blockIdx.x) / CG;             // tile walker index (pair index)
+    const int units = static_cast<int>(gridDim.x) / CG;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
+            mbar_init(&full_bar[s], 1);           // the (leader's) arrive.expect_tx
             mbar_init(&empty_bar[s], 1);
+        }
+        for (int j = 0; j < SF_RING; ++j) {
+            mbar_init(&sf_full_bar[j], CG);       // every scale producer of the unit
+            mbar_init(&sf_empty_bar[j], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull_bar[i], 1);
-            mbar_init(&tempty_bar[i], 4);
+            mbar_init(&tempty_bar[i], 4 * CG);    // every epilogue warp of the unit
         }
         mbar_init(drain_bar, 1);
         *s_abort = 0;
@@ -297,8 +371,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         tma_prefetch_desc(&p.tma_d);
     }
     if (warp == 1) {
-        tmem_alloc(s_tmem, Cfg::TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc<CG>(s_tmem, Cfg::TMEM_COLS);
+        tmem_relinquish<CG>();
     }
     if constexpr (KIND == kMasked) {
         // masked_m clamped to [0, max_m]; tile prefix over groups (warp 0 scans).
@@ -331,142 +405,206 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
+    const int kg_count = (p.kb + 3) / 4;
+    const int my_rows = BM * static_cast<int>(rank);  // this CTA's rows inside a tile
 
     if (warp == 0) {
-        // ------------------------------------------------------- producer --
-        const int kg_count = (p.kb + 3) / 4;
+        // -------------------------------------------------------- TMA producer --
+        [[maybe_unused]] uint32_t full_leader0 = 0;  // the leader's stage barriers (pairs)
+        if constexpr (CG == 2) full_leader0 = mapa_shared(smem_u32(&full_bar[0]), 0);
         int stage = 0;
         uint32_t phase = 0;
         int issued = 0;
-        int gcur = 0, gcur_ahead = 0;
-        Tile cur, ahead;
-        bool have = next_tile<KIND, true>(p, s_prefix, s_mm, blockIdx.x, gcur, cur, lane);
-        // Scale words of the next group to store. Their loads are issued one
-        // group (four stages) before they are needed, so the global-load
-        // latency hides behind the TMA traffic of those stages.
-        ScaleWords<BN, KIND> sw;
-        int ahead_t = blockIdx.x, ahead_kg = 0;
-        bool ahead_ok = have;
-        if (have) {
-            ahead = cur;
-            gcur_ahead = gcur;
-            sw.load(p, ahead, 0, lane);
-        }
+        int gcur = 0;
+        Tile cur;
         bool aborted = false;
-        for (int t = blockIdx.x; have; t += gridDim.x) {
-            const int b_row = cur.n_blk * BN;
+        for (int t = unit; !aborted && next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, cur, lane); t += units) {
+            const int a_row = cur.m_blk * BM * CG + my_rows;
+            const int b_row = cur.n_blk * BN + Cfg::B_ROWS * static_cast<int>(rank);
             const int g = max(cur.g, 0);
-            for (int kb = 0; kb < p.kb; ++kb) {
-                if (!wait_bounded(&empty_bar[stage], phase ^ 1u, p, s_abort)) { aborted = true; break; }
-                const bool sf_stage = (kb & 3) == 0;
-                if (lane == 0) {
-                    constexpr uint32_t bytes = Cfg::A_BYTES + Cfg::B_BYTES;
-                    if (sf_stage) mbar_expect_tx(&full_bar[stage], bytes);
-                    else mbar_arrive_expect_tx(&full_bar[stage], bytes);
+            for (int gi = 0; gi < kg_count && !aborted; ++gi) {
+            const int kgrp = rot_group(p, t, gi, kg_count);
+            for (int kb = 4 * kgrp; kb < min(4 * kgrp + 4, p.kb); ++kb) {
+                if (!wait_warp(&empty_bar[stage], phase ^ 1u, p, s_abort)) { aborted = true; break; }
+                if (elect_one()) {
                     uint8_t* a_dst = smem_a + stage * Cfg::A_BYTES;
                     uint8_t* b_dst = smem_b + stage * Cfg::B_BYTES;
                     const int kx = kb * BK;
-                    if constexpr (KIND == kMasked) {
-                        tma_load_3d(a_dst, &p.tma_a, &full_bar[stage], kx, cur.m_blk * BM, cur.g);
-                    } else {
-                        tma_load_2d(a_dst, &p.tma_a, &full_bar[stage], kx, cur.m_blk * BM);
-                    }
-                    if constexpr (KIND == kDense) {
-                        tma_load_2d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row);
-                    } else {
-                        tma_load_3d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row, g);
-                    }
-                }
-                if (sf_stage) {
-                    sw.store(smem_sfa + stage * Cfg::SFA_BYTES, smem_sfb + stage * Cfg::SFB_BYTES, lane);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    // test hook: CTA 0 withholds the arrive of its first stage
-                    const bool withhold = p.test_mode == 1 && blockIdx.x == 0 && issued == 0;
-                    if (lane == 0 && !withhold) mbar_arrive(&full_bar[stage]);
-                    // start the loads of the following group
-                    if (ahead_ok) {
-                        if (++ahead_kg == kg_count) {
-                            ahead_kg = 0;
-                            ahead_t += gridDim.x;
-                            ahead_ok = next_tile<KIND, true>(p, s_prefix, s_mm, ahead_t, gcur_ahead, ahead, lane);
+                    if constexpr (CG == 1) {
+                        mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
+                        if constexpr (KIND == kMasked) {
+                            tma_load_3d(a_dst, &p.tma_a, &full_bar[stage], kx, a_row, cur.g);
+                        } else {
+                            tma_load_2d(a_dst, &p.tma_a, &full_bar[stage], kx, a_row);
                         }
-                        if (ahead_ok) sw.load(p, ahead, ahead_kg, lane);
+                        if constexpr (KIND == kDense) {
+                            tma_load_2d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row);
+                        } else {
+                            tma_load_3d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row, g);
+                        }
+                    } else {
+                        // the leader arms its barrier for both CTAs' bytes; both
+                        // CTAs' loads complete on the leader's barrier
+                        if (leader) mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
+                        const uint32_t fb = full_leader0 + 8u * static_cast<uint32_t>(stage);
+                        tma_load_2d_pair(a_dst, &p.tma_a, fb, kx, a_row);
+                        tma_load_2d_pair(b_dst, &p.tma_b, fb, kx, b_row);
                     }
                 }
                 __syncwarp();
                 ++issued;
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
-            if (aborted) break;
-            have = next_tile<KIND, true>(p, s_prefix, s_mm, t + gridDim.x, gcur, cur, lane);
+            }
         }
         if (aborted) {
             // let the loads already issued land before shared memory goes away
-            int s = stage;
-            uint32_t ph = phase;
-            for (int i = 0; i < STAGES && i < issued; ++i) {
-                if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
-                wait_quiet(&full_bar[s], ph, p.wait_limit_ns / 16);
+            if constexpr (CG == 1) {
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && i < issued; ++i) {
+                    if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
+                    wait_quiet(&full_bar[s], ph, p.wait_limit_ns / 16);
+                }
+            } else {
+                sleep_ns(p.wait_limit_ns / 16);  // completion lands on the leader's barrier
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA --
-        constexpr uint32_t IDESC = idesc_mxf8_e4m3_ue8m0(BN);
-        int stage = 0;
-        uint32_t phase = 0;
-        int acc = 0;
-        uint32_t acc_phase = 0;
-        int gcur = 0;
-        Tile c;
+    } else if (warp == 6) {
+        // ------------------------------------------------------ scale producer --
+        [[maybe_unused]] uint32_t sf_full_leader0 = 0;  // the leader's scale barriers (pairs)
+        if constexpr (CG == 2) sf_full_leader0 = mapa_shared(smem_u32(&sf_full_bar[0]), 0);
+        int slot = 0;
+        uint32_t sf_phase = 0;
+        int groups_done = 0;
+        int gcur = 0, gcur_ahead = 0;
+        Tile cur, ahead;
+        bool have = next_tile<KIND, true>(p, s_prefix, s_mm, unit, gcur, cur, lane);
+        // The words of the next group are loaded one group ahead of their store.
+        ScaleWords<BN, KIND> sw;
+        int ahead_t = unit, ahead_kg = 0;
+        bool ahead_ok = have;
+        if (have) {
+            ahead = cur;
+            gcur_ahead = gcur;
+            sw.load(p, ahead.m_blk * BM * CG + my_rows, ahead.n_blk * BN, ahead.g, rot_group(p, unit, 0, kg_count), lane);
+        }
         bool aborted = false;
-        for (int t = blockIdx.x; !aborted && next_tile<KIND, false>(p, s_prefix, s_mm, t, gcur, c, lane); t += gridDim.x) {
-            if (!wait_bounded(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
-            for (int kb = 0; kb < p.kb; ++kb) {
-                if (!wait_bounded(&full_bar[stage], phase, p, s_abort)) { aborted = true; break; }
-                tc_fence_after();
-                if (lane == 0) {
-                    if ((kb & 3) == 0) {
-                        tc_cp_32x128b_warpx4(tmem_base + Cfg::SFA_COL,
-                                             smem_desc_sf(smem_u32(smem_sfa + stage * Cfg::SFA_BYTES)));
-#pragma unroll
-                        for (int ch = 0; ch < Cfg::SFB_CHUNKS; ++ch)
-                            tc_cp_32x128b_warpx4(tmem_base + Cfg::SFB_COL + 4 * ch,
-                                                 smem_desc_sf(smem_u32(smem_sfb + stage * Cfg::SFB_BYTES + 512 * ch)));
+        for (int t = unit; have && !aborted; t += units) {
+            for (int kg = 0; kg < kg_count; ++kg) {
+                if (!wait_bounded(&sf_empty_bar[slot], sf_phase ^ 1u, p, s_abort)) { aborted = true; break; }
+                uint8_t* sfa_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
+                sw.store(sfa_slot, sfa_slot + Cfg::SFA_BYTES, lane);
+                fence_proxy_async_smem();
+                __syncwarp();
+                // test hook: CTA 0 withholds the arrive of its first group
+                const bool withhold = p.test_mode == 1 && blockIdx.x == 0 && groups_done == 0;
+                if (lane == 0 && !withhold) {
+                    if (CG == 1 || leader) mbar_arrive(&sf_full_bar[slot]);
+                    else mbar_arrive_cluster_release(sf_full_leader0 + 8u * static_cast<uint32_t>(slot));
+                }
+                if (ahead_ok) {
+                    // start the loads of the following group
+                    if (++ahead_kg == kg_count) {
+                        ahead_kg = 0;
+                        ahead_t += units;
+                        ahead_ok = next_tile<KIND, true>(p, s_prefix, s_mm, ahead_t, gcur_ahead, ahead, lane);
                     }
-                    const uint32_t sf_id = static_cast<uint32_t>(kb & 3);
-                    const uint32_t idesc = idesc_with_sf_id(IDESC, sf_id);
-                    const uint32_t sfa_t = (tmem_base + Cfg::SFA_COL) | (sf_id << 30);
-                    const uint32_t sfb_t = (tmem_base + Cfg::SFB_COL) | (sf_id << 30);
-                    const uint64_t adesc = smem_desc_sw128(smem_u32(smem_a + stage * Cfg::A_BYTES));
-                    const uint64_t bdesc = smem_desc_sw128(smem_u32(smem_b + stage * Cfg::B_BYTES));
-#pragma unroll
-                    for (int k = 0; k < BK / MMA_K; ++k) {
-                        // advance the start address by 32 bytes of K inside the swizzled row
-                        const uint64_t koff = static_cast<uint64_t>((k * MMA_K) >> 4);
-                        tc_mma_mxf8f6f4_block_scale(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t, sfb_t,
-                                                    (kb > 0 || k > 0) ? 1u : 0u);
-                    }
-                    tc_commit(&empty_bar[stage]);
+                    if (ahead_ok)
+                        sw.load(p, ahead.m_blk * BM * CG + my_rows, ahead.n_blk * BN, ahead.g,
+                                rot_group(p, ahead_t, ahead_kg, kg_count), lane);
                 }
                 __syncwarp();
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                ++groups_done;
+                if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
             }
-            if (aborted) break;
-            if (lane == 0) tc_commit(&tfull_bar[acc]);
-            __syncwarp();
-            if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+            if (!aborted) have = next_tile<KIND, true>(p, s_prefix, s_mm, t + units, gcur, cur, lane);
         }
-        // all MMAs of this CTA must finish before TMEM is released
-        if (lane == 0) tc_commit(drain_bar);
-        __syncwarp();
+    } else if (warp == 1) {
+        // ----------------------------------------------------------------- MMA --
+        // The whole warp runs the loop and waits by vote; one lane, chosen by
+        // elect.sync, issues each batch of tcgen05.mma / cp / commit. Issuing
+        // from a converged warp keeps the tensor pipe fed: a loop run by a
+        // single lane (or guarded by a lane test) issues the same MMAs about a
+        // fifth slower per K-block on this part, because each barrier probe
+        // then stalls the issue of the MMAs that follow it.
+        if (leader) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int slot = 0;
+            uint32_t sf_phase = 0;
+            int acc = 0;
+            uint32_t acc_phase = 0;
+            int gcur = 0;
+            Tile c;
+            bool aborted = false;
+            uint32_t sf_tmem = tmem_base + Cfg::SF_BASE;
+            uint32_t sf_other = sf_tmem + Cfg::SF_COLS;
+            for (int t = unit; !aborted && next_tile<KIND, false>(p, s_prefix, s_mm, t, gcur, c, lane); t += units) {
+                if (!wait_warp(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
+                tc_fence_after();  // the epilogue's TMEM reads precede the MMAs below
+                const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
+                for (int gi = 0; gi < kg_count && !aborted; ++gi) {
+                    const int kgrp = rot_group(p, t, gi, kg_count);
+                    // this group's scale words (both CTAs of a pair) -> TMEM; the
+                    // slot is free again once the copy has completed
+                    const bool ok = (CG == 2) ? wait_warp<true>(&sf_full_bar[slot], sf_phase, p, s_abort)
+                                              : wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort);
+                    if (!ok) { aborted = true; break; }
+                    tc_fence_after();
+                    if (elect_one()) {
+                        const uint8_t* sf_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
+                        tc_cp_32x128b_warpx4<CG>(sf_tmem, smem_desc_sf(smem_u32(sf_slot)));
+#pragma unroll
+                        for (int ch = 0; ch < Cfg::SFB_CHUNKS; ++ch)
+                            tc_cp_32x128b_warpx4<CG>(sf_tmem + 4 + 4 * ch,
+                                                     smem_desc_sf(smem_u32(sf_slot + Cfg::SFA_BYTES + 512 * ch)));
+                        tc_commit<CG>(&sf_empty_bar[slot]);
+                    }
+                    __syncwarp();
+                    if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
+                    const uint32_t sf_cur = sf_tmem;
+                    sf_tmem = sf_other;
+                    sf_other = sf_cur;
+                    for (int kb = 4 * kgrp; kb < min(4 * kgrp + 4, p.kb); ++kb) {
+                        // TMA bytes observed complete on the barrier are visible to
+                        // the tensor core's shared-memory reads: no fence needed here
+                        if (!wait_warp(&full_bar[stage], phase, p, s_abort)) { aborted = true; break; }
+                        const uint32_t sf_id = static_cast<uint32_t>(kb & 3);
+                        const uint32_t idesc = idesc_with_sf_id(Cfg::IDESC, sf_id);
+                        const uint32_t sfa_t = sf_cur | (sf_id << 30);
+                        const uint32_t sfb_t = (sf_cur + 4) | (sf_id << 30);
+                        const uint64_t adesc = smem_desc_sw128(smem_u32(smem_a + stage * Cfg::A_BYTES));
+                        const uint64_t bdesc = smem_desc_sw128(smem_u32(smem_b + stage * Cfg::B_BYTES));
+                        if (elect_one()) {
+#pragma unroll
+                            for (int k = 0; k < BK / MMA_K; ++k) {
+                                // advance the start address by 32 bytes of K inside the swizzled row
+                                const uint64_t koff = static_cast<uint64_t>((k * MMA_K) >> 4);
+                                tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
+                                                                sfb_t, (gi > 0 || kb > 4 * kgrp || k > 0) ? 1u : 0u);
+                            }
+                            tc_commit<CG>(&empty_bar[stage]);
+                        }
+                        __syncwarp();
+                        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    }
+                }
+                if (aborted) break;
+                if (elect_one()) tc_commit<CG>(&tfull_bar[acc]);
+                __syncwarp();
+                if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+            }
+            // all MMAs must finish before TMEM is released (in both CTAs)
+            if (elect_one()) tc_commit<CG>(drain_bar);
+            __syncwarp();
+        }
         wait_quiet(drain_bar, 0, p.wait_limit_ns);
     } else {
-        // ------------------------------------------------------- epilogue --
+        // ------------------------------------------------------------ epilogue --
         // Each warp owns 32 rows (its TMEM sub-partition). Per tile it reads
         // the accumulator in batches of up to 128 columns, hands TMEM back to
         // the MMA warp right after the last read, and then writes bf16:
@@ -474,13 +612,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         // when all 32 rows may be written, predicated 16-byte stores otherwise.
         const int q = static_cast<int>(warp & 3);   // TMEM sub-partition of this warp
         uint8_t* stg = smem_epi + (warp - 2) * Cfg::EPI_WARP_BYTES;
+        [[maybe_unused]] uint32_t tempty_leader0 = 0;  // the leader's accumulator barriers (pairs)
+        if constexpr (CG == 2) tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
         int gcur = 0;
         int buf = 0;
         Tile c;
-        for (int t = blockIdx.x; next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, c, lane); t += gridDim.x) {
-            const int mloc = c.m_blk * BM + 32 * q + static_cast<int>(lane);
+        for (int t = unit; next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, c, lane); t += units) {
+            const int row_coord = c.m_blk * BM * CG + my_rows + 32 * q;
+            const int mloc = row_coord + static_cast<int>(lane);
             bool valid;
             size_t out_row;
             if constexpr (KIND == kDense) {
@@ -499,7 +640,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // TMA stores clip at the tensor's edges, so for the dense form rows
             // past M are safe; the grouped forms need every row of the chunk valid.
             const bool use_tma = (KIND == kDense) ? true : (__all_sync(0xffffffffu, valid) != 0);
-            const int row_coord = c.m_blk * BM + 32 * q;
             if (!wait_bounded(&tfull_bar[acc], acc_phase, p, s_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_COLS;
@@ -518,7 +658,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     // last TMEM read of this accumulator: hand it back to the MMA warp
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+                    if (lane == 0) {
+                        if (CG == 1 || leader) mbar_arrive(&tempty_bar[acc]);
+                        else mbar_arrive_cluster(tempty_leader0 + 8u * static_cast<uint32_t>(acc));
+                    }
                 }
 #pragma unroll
                 for (int j = 0; j < kMaxBatch / 32; ++j) {
@@ -570,9 +713,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (CG == 2) cluster_sync();  // neither CTA frees TMEM while the pair still uses it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+        tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);
     }
 }
 

@@ -1,7 +1,7 @@
 """Run one GEMM form a few times on seeded inputs: a small, self-contained case
 for profilers (e.g. ncu) and quick timing.
 
-    python -m moe_grouped_gemm_tcgen05_b200.profile_case dense --m 4096 --n 7168 --k 16384 --iters 3
+    python -m moe_grouped_gemm_tcgen05_b200.profile_case dense --m 4096 --n 7168 --k 16384 --iters 3 [--cta-group 2]
     python -m moe_grouped_gemm_tcgen05_b200.profile_case masked --groups 32 --max-m 256 --expected-m 96 --n 4096 --k 7168
     python -m moe_grouped_gemm_tcgen05_b200.profile_case contiguous --groups 8 --n 4096 --k 7168
 
@@ -32,11 +32,13 @@ def main(argv=None):
     ap.add_argument("--expected-m", type=int, default=96)
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--block-n", type=int, default=0)
+    ap.add_argument("--cta-group", type=int, default=0, help="dense only: 1 = single CTAs, 2 = CTA pairs")
     args = ap.parse_args(argv)
 
     torch.cuda.set_device(0)
     dg.init()
     dg.set_block_n(args.block_n)
+    dg.set_cta_group(args.cta_group)
     if args.form == "dense":
         p = W.dense_t(args.m, args.n, args.k, seed=1001)
         sfa, sfb = dg.pack_ue8m0(p["sfa_f32"]), dg.pack_ue8m0(p["sfb_f32"])

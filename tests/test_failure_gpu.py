@@ -34,15 +34,16 @@ def _masked(q):
     return d
 
 
-@pytest.mark.parametrize("form", ["dense", "masked"])
+@pytest.mark.parametrize("form", ["dense", "dense_pairs", "masked"])
 def test_timeout_is_reported_and_context_survives(form):
     dg.init()
     dg.device_error(clear=True)
+    dg.set_cta_group(2 if form == "dense_pairs" else 0)
     p = W.dense(384, 512, 1024, seed=31)
     q = W.masked(np.array([100, 0, 256], dtype=np.int32), 256, 256, 512, seed=32)
     try:
         dg.set_test_hooks(1, 200)
-        _dense(p) if form == "dense" else _masked(q)
+        _masked(q) if form == "masked" else _dense(p)
         torch.cuda.synchronize()
         assert dg.device_error(clear=True) & dg.DEVERR_TIMEOUT
     finally:
@@ -59,3 +60,4 @@ def test_timeout_is_reported_and_context_survives(form):
         oracle.pack_ue8m0(q["sfb_f32"].reshape(-1, 4)).reshape(3, 2, 1), q["masked_m"])
     check_fp(bf16_to_f64(dm)[valid], refm[valid], "masked after timeout")
     assert dg.device_error(clear=True) == 0
+    dg.set_cta_group(0)

@@ -24,6 +24,7 @@ def _reset():
     dg.device_error(clear=True)
     yield
     dg.set_block_n(0)
+    dg.set_cta_group(0)
     assert dg.device_error(clear=True) & dg.DEVERR_TIMEOUT == 0
 
 
@@ -39,8 +40,9 @@ def _oracle_pack(sf_f32):
     return oracle.pack_ue8m0(sf_f32.reshape(-1, sf_f32.shape[-1])).reshape(*sf_f32.shape[:-1], -1)
 
 
-def run_dense(p, bn=0):
+def run_dense(p, bn=0, cg=0):
     dg.set_block_n(bn)
+    dg.set_cta_group(cg)
     d = torch.empty((p["M"], p["N"]), dtype=torch.bfloat16, device="cuda")
     fill_sentinel(d)
     dg.fp8_gemm_nt(_dev(p["a"]), _pack_dev(p["sfa_f32"]), _dev(p["b"]), _pack_dev(p["sfb_f32"]), d)
@@ -59,6 +61,20 @@ def test_dense_parity_every_tile_width(bn, mnk):
     d = run_dense(p, bn)
     assert not is_sentinel(d).any()
     check_fp(bf16_to_f64(d), ref_dense(p), f"dense {mnk} bn={bn}")
+
+
+PAIR_BLOCK_NS = [128, 160, 192, 224, 256]
+
+
+@pytest.mark.parametrize("bn", PAIR_BLOCK_NS)
+@pytest.mark.parametrize("mnk", [(300, 400, 1024), (512, 256, 512), (257, 264, 640), (1024, 1000, 2048)])
+def test_dense_parity_cta_pairs(bn, mnk):
+    # 256-row tiles on CTA pairs; M not a multiple of 256 leaves the odd CTA
+    # of the last pair partly or wholly past M
+    p = W.dense(*mnk, seed=3 * sum(mnk))
+    d = run_dense(p, bn, cg=2)
+    assert not is_sentinel(d).any()
+    check_fp(bf16_to_f64(d), ref_dense(p), f"dense pairs {mnk} bn={bn}")
 
 
 @pytest.mark.parametrize("mnk", [(1, 16, 128), (64, 2112, 896), (128, 8, 128), (513, 1000, 2048)])
@@ -89,12 +105,12 @@ def _pack_bytes_host(byts):
     return w.astype(np.uint32).view(np.int32)
 
 
-@pytest.mark.parametrize("bn", BLOCK_NS)
-def test_one_hot_rows_are_bit_exact(bn):
+@pytest.mark.parametrize("bn,cg", [(b, 1) for b in BLOCK_NS] + [(b, 2) for b in PAIR_BLOCK_NS])
+def test_one_hot_rows_are_bit_exact(bn, cg):
     # one-hot A rows with power-of-two scales: every output is a single product
     # e4m3 * 2^a * 2^b, exactly representable in bf16
     rng = np.random.default_rng(bn)
-    M, N, K = 200, 304, 1152
+    M, N, K = 300, 304, 1152
     KB = K // 128
     ks = rng.integers(0, K, size=M)
     a = np.zeros((M, K), dtype=np.uint8)
@@ -104,6 +120,7 @@ def test_one_hot_rows_are_bit_exact(bn):
     b = _codes(rng, (N, K))
     sfa, sfb = _pack_bytes_host(ea), _pack_bytes_host(eb)
     dg.set_block_n(bn)
+    dg.set_cta_group(cg)
     d = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
     dg.fp8_gemm_nt(_dev(a), _dev(sfa), _dev(b), _dev(sfb), d)
     want = oracle.fp8_gemm_nt(a, sfa, b, sfb)
