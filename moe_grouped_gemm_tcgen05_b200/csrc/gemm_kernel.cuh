@@ -12,8 +12,8 @@
 //               into a STAGES-deep shared-memory ring.
 //   warp 6      scale producer: per group of four K-blocks (one packed int32
 //               per row/column) gathers the scale words into the 32x16-byte
-//               layout that tcgen05.cp expects, into its own 4-deep ring,
-//               loads issued one group ahead.
+//               layout that tcgen05.cp expects, into its own 4-deep ring, with
+//               the loads of the next two groups in flight.
 //   warp 1      MMA issuer: allocates TMEM, copies each group's scale words to
 //               TMEM (and frees their slot as soon as the copy completes),
 //               issues tcgen05.mma.kind::mxf8f6f4.block_scale (K=32) four
@@ -27,6 +27,11 @@
 //               rows that must not be written (past masked_m, padding of
 //               m_indices) use predicated row stores instead, so those rows
 //               are never touched.
+// Every role runs its loop on the whole warp: waits are warp-wide votes and
+// the TMA / tcgen05 instructions are issued by one lane chosen with
+// elect.sync. (A loop run by one lane, or guarded by a lane test, leaves the
+// tensor pipe idle for part of every K-block: each barrier probe then holds up
+// the MMAs issued after it.)
 // The accumulator is double-buffered in TMEM when two fit next to the scale
 // columns, so the epilogue of tile i overlaps the MMAs of tile i+1.
 //
@@ -34,12 +39,15 @@
 // a 256 x BN tile whose A rows are split 128/128 and whose B rows are split
 // BN/2 / BN/2 between the two CTAs' shared memory. Only the even CTA (the
 // leader) issues MMAs and tcgen05 copies (all with cta_group::2); both CTAs'
-// TMA loads complete on the leader's stage barrier, the odd CTA publishes its
-// scale words with a cluster-scope release on the leader's scale barrier
-// (the scale ring gives that release several groups of slack), and commits
-// reach both CTAs' barriers. Each CTA's TMEM holds its 128 rows x BN of the
+// TMA loads complete on the leader's stage barrier, the leader's scale warp
+// gathers both CTAs' scale words and writes the peer's share into the peer's
+// shared memory (so that hand-off stays inside the leader), and commits reach
+// both CTAs' barriers. Each CTA's TMEM holds its 128 rows x BN of the
 // accumulator, its own A scales and the full-width B scales. Per SM this
-// halves the B bytes each 128-K block needs. No load is multicast.
+// halves the B bytes each 128-K block needs, which is what bounds a single
+// CTA: the L2 feeds an SM about 77 bytes per clock, so a 128 x 224 tile
+// (44 KB per K-block) waits on loads while a pair's 30 KB per SM does not.
+// No load is multicast.
 //
 // Block scaling: the hardware MMA applies one UE8M0 scale per 32 K values for
 // each row of A and each column of B. The 128-granular scales of this format
@@ -144,35 +152,14 @@ __device__ __forceinline__ uint64_t global_ns() {
     return t;
 }
 
-// Wait for the phase of `bar` with the given parity. Gives up when another
-// role of this CTA has given up, or after p.wait_limit_ns; a timeout is
-// recorded in the device status word.
-// CLUSTER_ACQUIRE: the phase publishes shared-memory data written by the peer
-// CTA of a pair (its scale words), so the probe acquires at cluster scope.
-template <bool CLUSTER_ACQUIRE = false>
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const GemmParams& p,
-                                             volatile int* s_abort) {
-    auto probe = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
-    if (probe()) return true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-        if (probe()) return true;
-        if (*s_abort) return false;
-        if (global_ns() - t0 > p.wait_limit_ns) {
-            atomicOr(p.status, DEVERR_TIMEOUT);
-            *s_abort = 1;
-            return false;
-        }
-    }
-}
-
-// Warp-wide form of wait_bounded: every lane probes and the outcome is a vote,
-// so all 32 lanes leave together with the same answer. Roles that issue
-// tcgen05 instructions under elect.sync use it: a lane that left a loop early
-// would leave the others waiting at the next elect.sync.
-template <bool CLUSTER_ACQUIRE = false>
+// Wait for the phase of `bar` with the given parity, as a whole warp: every
+// lane probes and the outcome is a vote, so all 32 lanes leave together with
+// the same answer (a lane that left a loop early would leave the others
+// waiting at the next elect.sync, __syncwarp or .sync.aligned instruction).
+// Gives up when another role of this CTA has given up, or after
+// p.wait_limit_ns; a timeout is recorded in the device status word.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const GemmParams& p, volatile int* s_abort) {
-    auto probe = [&]() { return CLUSTER_ACQUIRE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+    auto probe = [&]() { return mbar_try_wait(bar, parity); };
     if (__all_sync(0xffffffffu, probe())) return true;
     const uint64_t t0 = global_ns();
     while (true) {
@@ -272,15 +259,17 @@ __device__ __forceinline__ int rot_group(const GemmParams& p, int t, int gi, int
 
 // ------------------------------------------------------- scale-word gather --
 
-// Scale words of one 4-K-block group for this CTA's part of a tile: lane r
-// holds, for j = 0..3, the word of A row row0 + 32j + r and, per 128-column
-// chunk, the word of B column n0 + 128*chunk + 32j + r. Stored as one 16-byte
-// row per lane, this is the 32x128-bit matrix whose copy to TMEM puts row m at
-// lane m % 32, column m / 32.
-template <int BN, int KIND>
+// Scale words of one 4-K-block group of a tile: lane r holds, for j = 0..3,
+// the word of A row row0 + 32j + r and, per 128-column chunk, the word of B
+// column n0 + 128*chunk + 32j + r. Stored as one 16-byte row per lane, this is
+// the 32x128-bit matrix whose copy to TMEM puts row m at lane m % 32, column
+// m / 32. For a CTA pair (CG = 2) the words of the second CTA's 128 rows are
+// gathered too (`ap`), by the leader, which stores them into the peer's slot.
+template <int BN, int KIND, int CG>
 struct ScaleWords {
     static constexpr int CH = (BN + 127) / 128;
     uint32_t a[4];
+    uint32_t ap[CG == 2 ? 4 : 1];
     uint32_t b[CH][4];
 
     __device__ __forceinline__ void load(const GemmParams& p, int row0, int n0, int g, int kg, uint32_t lane) {
@@ -292,6 +281,10 @@ struct ScaleWords {
         for (int j = 0; j < 4; ++j) {
             const int r = min(row0 + 32 * j + static_cast<int>(lane), p.rows - 1);
             a[j] = static_cast<uint32_t>(__ldg(p.sfa + (row_base + r) * p.kp + kg));
+            if constexpr (CG == 2) {
+                const int rp = min(row0 + BM + 32 * j + static_cast<int>(lane), p.rows - 1);
+                ap[j] = static_cast<uint32_t>(__ldg(p.sfa + (row_base + rp) * p.kp + kg));
+            }
         }
         const int32_t* sfb = p.sfb + static_cast<size_t>(KIND == kDense ? 0 : max(g, 0)) * p.nb_sf * p.kp;
 #pragma unroll
@@ -310,6 +303,17 @@ struct ScaleWords {
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch)
             reinterpret_cast<uint4*>(sfb_slot + 512 * ch)[lane] = make_uint4(b[ch][0], b[ch][1], b[ch][2], b[ch][3]);
+    }
+
+    // The peer CTA's copy of the slot (pairs): its A rows and the same B words,
+    // written through the cluster window at the same shared-memory offsets.
+    __device__ __forceinline__ void store_peer(uint32_t sfa_slot_peer, uint32_t sfb_slot_peer, uint32_t lane) const {
+        if constexpr (CG == 2) {
+            st_cluster_v4(sfa_slot_peer + 16u * lane, ap[0], ap[1], ap[2], ap[3]);
+#pragma unroll
+            for (int ch = 0; ch < CH; ++ch)
+                st_cluster_v4(sfb_slot_peer + 512u * ch + 16u * lane, b[ch][0], b[ch][1], b[ch][2], b[ch][3]);
+        }
     }
 };
 
@@ -354,7 +358,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             mbar_init(&empty_bar[s], 1);
         }
         for (int j = 0; j < SF_RING; ++j) {
-            mbar_init(&sf_full_bar[j], CG);       // every scale producer of the unit
+            mbar_init(&sf_full_bar[j], 1);        // the scale producer (the leader's, for a pair)
             mbar_init(&sf_empty_bar[j], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -475,53 +479,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         }
     } else if (warp == 6) {
         // ------------------------------------------------------ scale producer --
-        [[maybe_unused]] uint32_t sf_full_leader0 = 0;  // the leader's scale barriers (pairs)
-        if constexpr (CG == 2) sf_full_leader0 = mapa_shared(smem_u32(&sf_full_bar[0]), 0);
-        int slot = 0;
-        uint32_t sf_phase = 0;
-        int groups_done = 0;
-        int gcur = 0, gcur_ahead = 0;
-        Tile cur, ahead;
-        bool have = next_tile<KIND, true>(p, s_prefix, s_mm, unit, gcur, cur, lane);
-        // The words of the next group are loaded one group ahead of their store.
-        ScaleWords<BN, KIND> sw;
-        int ahead_t = unit, ahead_kg = 0;
-        bool ahead_ok = have;
-        if (have) {
-            ahead = cur;
-            gcur_ahead = gcur;
-            sw.load(p, ahead.m_blk * BM * CG + my_rows, ahead.n_blk * BN, ahead.g, rot_group(p, unit, 0, kg_count), lane);
-        }
-        bool aborted = false;
-        for (int t = unit; have && !aborted; t += units) {
-            for (int kg = 0; kg < kg_count; ++kg) {
-                if (!wait_bounded(&sf_empty_bar[slot], sf_phase ^ 1u, p, s_abort)) { aborted = true; break; }
+        // For a pair the leader's warp gathers the words of both CTAs and writes
+        // the peer's share into the peer's shared memory, so the hand-off to the
+        // MMA warp stays inside the leader CTA; the peer's warp has no work.
+        if (CG == 1 || leader) {
+            [[maybe_unused]] uint32_t peer_sf0 = 0;  // the peer's scale ring (pairs)
+            if constexpr (CG == 2) peer_sf0 = mapa_shared(smem_u32(smem_sf), 1);
+            // Groups are visited in the MMA warp's order (tile by tile, K groups
+            // in order). Two register sets keep the loads of two groups in
+            // flight while a third is stored.
+            int ct = unit, ckg = 0, cg_cur = 0;
+            Tile ctile;
+            bool cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+            auto load_next = [&](ScaleWords<BN, KIND, CG>& w) -> bool {
+                if (!cok) return false;
+                w.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, rot_group(p, ct, ckg, kg_count), lane);
+                if (++ckg == kg_count) {
+                    ckg = 0;
+                    ct += units;
+                    cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+                }
+                return true;
+            };
+            int slot = 0;
+            uint32_t sf_phase = 0;
+            int groups_done = 0;
+            // store one group into the next ring slot and publish it; false on abort
+            auto put = [&](const ScaleWords<BN, KIND, CG>& w) -> bool {
+                if (!wait_warp(&sf_empty_bar[slot], sf_phase ^ 1u, p, s_abort)) return false;
                 uint8_t* sfa_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
-                sw.store(sfa_slot, sfa_slot + Cfg::SFA_BYTES, lane);
-                fence_proxy_async_smem();
+                w.store(sfa_slot, sfa_slot + Cfg::SFA_BYTES, lane);
+                if constexpr (CG == 2) {
+                    const uint32_t peer_slot = peer_sf0 + static_cast<uint32_t>(slot * Cfg::SF_SLOT_BYTES);
+                    w.store_peer(peer_slot, peer_slot + Cfg::SFA_BYTES, lane);
+                    fence_proxy_async_cluster();  // remote generic stores -> the async proxy (tcgen05.cp)
+                } else {
+                    fence_proxy_async_smem();
+                }
                 __syncwarp();
                 // test hook: CTA 0 withholds the arrive of its first group
                 const bool withhold = p.test_mode == 1 && blockIdx.x == 0 && groups_done == 0;
-                if (lane == 0 && !withhold) {
-                    if (CG == 1 || leader) mbar_arrive(&sf_full_bar[slot]);
-                    else mbar_arrive_cluster_release(sf_full_leader0 + 8u * static_cast<uint32_t>(slot));
-                }
-                if (ahead_ok) {
-                    // start the loads of the following group
-                    if (++ahead_kg == kg_count) {
-                        ahead_kg = 0;
-                        ahead_t += units;
-                        ahead_ok = next_tile<KIND, true>(p, s_prefix, s_mm, ahead_t, gcur_ahead, ahead, lane);
-                    }
-                    if (ahead_ok)
-                        sw.load(p, ahead.m_blk * BM * CG + my_rows, ahead.n_blk * BN, ahead.g,
-                                rot_group(p, ahead_t, ahead_kg, kg_count), lane);
-                }
+                if (lane == 0 && !withhold) mbar_arrive(&sf_full_bar[slot]);
                 __syncwarp();
                 ++groups_done;
                 if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
+                return true;
+            };
+            ScaleWords<BN, KIND, CG> w0, w1;
+            bool v0 = load_next(w0);
+            bool v1 = load_next(w1);
+            while (v0) {
+                if (!put(w0)) break;
+                v0 = load_next(w0);
+                if (!v1) break;
+                if (!put(w1)) break;
+                v1 = load_next(w1);
             }
-            if (!aborted) have = next_tile<KIND, true>(p, s_prefix, s_mm, t + units, gcur, cur, lane);
         }
     } else if (warp == 1) {
         // ----------------------------------------------------------------- MMA --
@@ -551,9 +564,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     const int kgrp = rot_group(p, t, gi, kg_count);
                     // this group's scale words (both CTAs of a pair) -> TMEM; the
                     // slot is free again once the copy has completed
-                    const bool ok = (CG == 2) ? wait_warp<true>(&sf_full_bar[slot], sf_phase, p, s_abort)
-                                              : wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort);
-                    if (!ok) { aborted = true; break; }
+                    if (!wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort)) { aborted = true; break; }
                     tc_fence_after();
                     if (elect_one()) {
                         const uint8_t* sf_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
@@ -640,7 +651,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // TMA stores clip at the tensor's edges, so for the dense form rows
             // past M are safe; the grouped forms need every row of the chunk valid.
             const bool use_tma = (KIND == kDense) ? true : (__all_sync(0xffffffffu, valid) != 0);
-            if (!wait_bounded(&tfull_bar[acc], acc_phase, p, s_abort)) break;
+            if (!wait_warp(&tfull_bar[acc], acc_phase, p, s_abort)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_COLS;
             const int n0 = c.n_blk * BN;
