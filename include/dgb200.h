@@ -117,8 +117,8 @@ DG_API dg_status dgb200_set_cta_group(int cta_group);
 /*
  * Test hook for the failure path (process-wide). wait_limit_ms bounds every
  * wait inside the GEMM kernels (0 restores the default, 2000 ms). mode 1 makes
- * CTA 0 of each GEMM launch withhold the arrive of its first pipeline stage,
- * so a wait runs out: that launch leaves its output incomplete, sets
+ * CTA 0 of each GEMM launch withhold the arrive that publishes its first group
+ * of scale words, so a wait runs out: that launch leaves its output incomplete, sets
  * DG_DEVERR_TIMEOUT and returns; the CUDA context stays usable. mode 0 is
  * normal operation.
  */

@@ -101,7 +101,7 @@ struct GemmParams {
     int raster_group;         // m-tiles per raster band (dense / contiguous)
     uint64_t wait_limit_ns;   // bound of every mbarrier wait
     int k_rotate;             // 1: each tile walks its K groups starting at group (tile mod groups)
-    int test_mode;            // 1: CTA 0 withholds one stage arrive (exercises the timeout path)
+    int test_mode;            // 1: CTA 0 withholds its first scale-group arrive (exercises the timeout path)
 };
 
 template <int BN, int CG, bool SCHED_SMEM>
