@@ -115,6 +115,26 @@ DG_API int dgb200_block_n_supported(int block_n);
 DG_API dg_status dgb200_set_cta_group(int cta_group);
 
 /*
+ * Split-K for the dense GEMM (process-wide; tests and tuning). 0 restores the
+ * heuristic, which splits K only when the output tiles alone leave SMs idle
+ * (small M). 1 never splits. s >= 2 splits every dense call into s ranges of
+ * whole K groups (four 128-K blocks each; with G groups, range i covers groups
+ * [i*G/s, (i+1)*G/s)); a combination that is not possible (s larger than G,
+ * CTA pairs forced, workspace too small) makes the dense call return
+ * DG_ERR_UNSUPPORTED.
+ * A split unit writes its fp32 partial tile to a workspace that the library
+ * allocates (40 MB, with 4096 per-tile counters) when it first sets up the
+ * device. The last unit to finish a tile adds the partials in split order
+ * (the same result whichever unit is last) and writes the bf16 tile. The
+ * counters return to zero by themselves; after a launch that gave up
+ * (DG_DEVERR_TIMEOUT), dgb200_device_error(bits, 1) zeroes them again. Calls
+ * that may split must not run concurrently on two streams of one device (they
+ * share the workspace).
+ * Returns DG_ERR_UNSUPPORTED for s outside [0, 16].
+ */
+DG_API dg_status dgb200_set_splits(int splits);
+
+/*
  * Test hook for the failure path (process-wide). wait_limit_ms bounds every
  * wait inside the GEMM kernels (0 restores the default, 2000 ms). mode 1 makes
  * CTA 0 of each GEMM launch withhold the arrive that publishes its first group

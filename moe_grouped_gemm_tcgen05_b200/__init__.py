@@ -23,7 +23,7 @@ import torch
 __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-    "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group",
+    "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -78,6 +78,8 @@ def load():
         L.dgb200_block_n_supported.argtypes = [i32]
         L.dgb200_set_cta_group.restype = i32
         L.dgb200_set_cta_group.argtypes = [i32]
+        L.dgb200_set_splits.restype = i32
+        L.dgb200_set_splits.argtypes = [i32]
         L.dgb200_set_test_hooks.restype = i32
         L.dgb200_set_test_hooks.argtypes = [i32, i32]
         L.fp8_gemm_nt.restype = i32
@@ -147,9 +149,15 @@ def set_cta_group(cta_group: int):
     _check("dgb200_set_cta_group", load().dgb200_set_cta_group(int(cta_group)))
 
 
+def set_splits(splits: int):
+    """Split-K for the dense GEMM: 0 = heuristic, 1 = never, s >= 2 = s ranges of K."""
+    _check("dgb200_set_splits", load().dgb200_set_splits(int(splits)))
+
+
 def set_test_hooks(mode: int = 0, wait_limit_ms: int = 0):
-    """Failure-path test hook: mode 1 withholds one pipeline arrive in CTA 0 so
-    that a bounded wait runs out (see include/dgb200.h). mode 0 = normal."""
+    """Failure-path test hook: mode 1 makes CTA 0 withhold the arrive of its
+    first group of scale words so that a bounded wait runs out (see
+    include/dgb200.h). mode 0 = normal."""
     _check("dgb200_set_test_hooks", load().dgb200_set_test_hooks(int(mode), int(wait_limit_ms)))
 
 

@@ -3,8 +3,10 @@
 // Each compute call validates its scalars and pointers on the host, encodes
 // the TMA tensor maps (driver entry point, no libcuda link), picks a tile
 // width from the sizes and the SM count, and launches one kernel on the
-// caller's stream. Nothing here allocates device memory, synchronises, or reads
-// a device value, so every compute call can be captured in a CUDA Graph.
+// caller's stream. A compute call allocates nothing, never synchronises and
+// reads no device value, so it can be captured in a CUDA Graph. Device memory
+// is allocated once per device, when the library first sets that device up:
+// the split-K workspace (partial tiles and per-tile counters).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -29,11 +31,18 @@ using dg::GemmParams;
 
 constexpr int kMaxDevices = 64;
 
+// Split-K workspace per device: fp32 partial tiles and one counter per output
+// tile. Sized for up to two waves of 128 x 256 partials over the SMs.
+constexpr size_t kSplitWsBytes = size_t(40) << 20;
+constexpr int kSplitCounters = 4096;
+
 struct DeviceState {
     bool ready = false;
     int sms = 0;
     uint32_t* status = nullptr;  // address of g_dg_device_status on this device
     int max_pairs[64] = {};      // co-resident CTA pairs per kernel entry (cluster kernels only)
+    float* split_ws = nullptr;   // split-K partials (null: split-K disabled on this device)
+    uint32_t* split_counters = nullptr;
 };
 
 std::mutex g_mu;
@@ -41,6 +50,7 @@ DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_bn{0};
 std::atomic<int> g_force_cg{0};
+std::atomic<int> g_force_splits{0};
 std::atomic<int> g_test_mode{0};
 std::atomic<uint64_t> g_wait_limit_ns{dg::DEFAULT_WAIT_LIMIT_NS};
 // DGB200_LOG=1 in the environment prints each GEMM launch's configuration to stderr.
@@ -67,10 +77,12 @@ struct KernelEntry {
     int cg;     // CTAs per MMA unit (1, or a cluster pair)
     void* fn;
     int smem;
+    int stages;  // depth of the operand ring
 };
 
-#define DG_ENTRY(BN, KIND, CG) \
-    {BN, KIND, CG, kernel_ptr<BN, KIND, CG>(), dg::GemmConfig<BN, CG, KIND == dg::kMasked>::SMEM_BYTES}
+#define DG_ENTRY(BN, KIND, CG)                                                                 \
+    {BN, KIND, CG, kernel_ptr<BN, KIND, CG>(), dg::GemmConfig<BN, CG, KIND == dg::kMasked>::SMEM_BYTES, \
+     dg::GemmConfig<BN, CG, KIND == dg::kMasked>::STAGES}
 #define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1)
 
 const KernelEntry kKernels[] = {
@@ -129,6 +141,19 @@ dg_status init_device(int dev) {
     void* status = nullptr;
     if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
     st.status = static_cast<uint32_t*>(status);
+    // split-K workspace: optional; without it the GEMMs run unsplit
+    void* ws = nullptr;
+    void* ctr = nullptr;
+    if (cudaMalloc(&ws, kSplitWsBytes) == cudaSuccess &&
+        cudaMalloc(&ctr, kSplitCounters * sizeof(uint32_t)) == cudaSuccess &&
+        cudaMemset(ctr, 0, kSplitCounters * sizeof(uint32_t)) == cudaSuccess) {
+        st.split_ws = static_cast<float*>(ws);
+        st.split_counters = static_cast<uint32_t*>(ctr);
+    } else {
+        if (ws) cudaFree(ws);
+        if (ctr) cudaFree(ctr);
+        cudaGetLastError();  // clear the allocation error; split-K stays off
+    }
     st.ready = true;
     return DG_OK;
 }
@@ -180,13 +205,31 @@ constexpr double kL2BytesPerClk = 77.0;
 // Tensor-core clocks lost per tile when the accumulator is single-buffered
 // (the MMA warp waits for the epilogue's TMEM reads).
 constexpr double kSingleBufferBubble = 600.0;
+// Fewest clocks per block-scaled MMA issued from the MMA warp (small N).
+constexpr double kMinMmaClocks = 98.0;
+// HBM bytes per SM clock for the whole GPU (~6.5 TB/s at ~1.85 GHz).
+constexpr double kHbmBytesPerClk = 3500.0;
+// When each B tile is read once (a single m-tile: small M), the weights stream
+// from HBM as 128-byte pieces of many rows. Measured on B200: a CTA keeps at
+// most `stages` K-blocks in flight and each takes ~2.4 us (4400 clocks) from
+// issue to arrival; all CTAs together draw about 2400 bytes per clock.
+constexpr double kHbmLatencyClk = 4400.0;
+constexpr double kBStreamBytesPerClk = 2400.0;
+// Split-K: the most ranges per tile; the unit that reduces a tile pays about
+// one L2 round trip (~700 clocks) per 32 columns per two splits, plus a fixed
+// hand-off (fence, counter) of ~2000 clocks.
+constexpr int kMaxSplits = 16;
+constexpr double kL2LatencyClk = 700.0;
+constexpr double kSplitFixedClocks = 2000.0;
 
 // Clocks one SM spends per 128-K block of its (rows_a x bn) share of a tile:
 // the larger of the tensor core (four K=32 block-scaled MMAs of bn/2 clocks
-// each; a pair's MMA covers 128 rows on each of its two SMs) and the L2 feed
-// of the stage (rows_a rows of A and bn/cg rows of B, 128 bytes each).
+// each, but no less than ~98 clocks per MMA issued; a pair's MMA covers 128
+// rows on each of its two SMs) and the L2 feed of the stage (rows_a rows of A
+// and bn/cg rows of B, 128 bytes each).
 double kblock_clocks(int bn, int cg, int rows_a) {
-    const double tc = 2.0 * bn;
+    const double per_mma = bn / 2.0 > kMinMmaClocks ? bn / 2.0 : kMinMmaClocks;
+    const double tc = 4.0 * per_mma;
     const double l2 = (rows_a + static_cast<double>(bn) / cg) * 128.0 / kL2BytesPerClk;
     return tc > l2 ? tc : l2;
 }
@@ -195,16 +238,26 @@ int num_acc_for(int bn) { return (2 * bn + 2 * (4 + 4 * ((bn + 127) / 128)) <= 5
 
 struct TileChoice {
     const KernelEntry* entry;
-    int units;  // concurrent MMA units (CTAs, or CTA pairs)
+    int units;             // concurrent MMA units (CTAs, or CTA pairs)
+    int splits;            // split-K ranges per output tile (1 = none)
 };
 
-// Pick the kernel (N tile, one CTA or a CTA pair) with the least modelled
-// time: waves of tiles over the concurrent MMA units x time per tile.
-TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int kb, long long m128_blocks) {
+// Pick the kernel (N tile, one CTA or a CTA pair) and, for the dense form,
+// the split-K factor with the least modelled time: waves of work units over
+// the concurrent MMA units x time per unit, but no less than the problem's
+// unique bytes at the HBM rate. Split-K is considered only when the output
+// tiles alone leave SMs idle; a split unit also pays for writing its fp32
+// partial and, on average, for one reduction read of all partials.
+TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
+                       long long unique_bytes) {
+    const int kb = k / 128;
+    const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
     const int forced_cg = kind == dg::kDense ? g_force_cg.load() : 0;  // pairs exist for the dense form only
-    TileChoice best{nullptr, 0};
+    const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
+    TileChoice best{nullptr, 0, 1};
     double best_cost = 1e300;
+    const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
         if (e.kind != kind) continue;
@@ -215,17 +268,44 @@ TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int kb,
         if (units < 1) continue;
         const long long mt = (m128_blocks + e.cg - 1) / e.cg;
         const long long nb = (n + e.bn - 1) / e.bn;
-        const long long waves = (mt * nb + units - 1) / units;
+        const long long tiles = mt * nb;
         const int rows_a = rows < dg::BM ? rows : dg::BM;
-        const double tile =
-            kb * kblock_clocks(e.bn, e.cg, rows_a) + (num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0);
-        const double cost = static_cast<double>(waves) * tile;
-        const bool better = cost < best_cost * 0.999 ||
-                            (cost <= best_cost * 1.001 && best.entry && (e.cg > best.entry->cg ||
-                                                                         (e.cg == best.entry->cg && e.bn > best.entry->bn)));
-        if (best.entry == nullptr || better) {
-            best_cost = cost;
-            best = TileChoice{&e, units};
+        const double kbc0 = kblock_clocks(e.bn, e.cg, rows_a);
+        const double bubble = num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0;
+        for (int splits = 1; splits <= kMaxSplits; ++splits) {
+            if (forced_splits != 0 && splits != forced_splits) continue;
+            const bool can_split = kind == dg::kDense && e.cg == 1 && st->split_ws != nullptr;
+            if (splits > 1) {
+                if (!can_split || splits > kg) break;
+                if (forced_splits == 0 && tiles >= units) break;  // the tiles alone fill the GPU
+                if (tiles > kSplitCounters) break;
+                if (static_cast<double>(tiles) * splits * dg::BM * e.bn * sizeof(float) > kSplitWsBytes) break;
+            }
+            const int gps = (kg + splits - 1) / splits;  // K groups of the longest range
+            const long long work = tiles * splits;
+            const long long waves = (work + units - 1) / units;
+            const int kb_unit = gps * 4 < kb ? gps * 4 : kb;
+            double kbc = kbc0;
+            if (mt == 1) {  // B streamed once from HBM
+                const double active = static_cast<double>(work < units ? work : units);
+                const double lat = kHbmLatencyClk / e.stages;
+                const double bw = static_cast<double>(e.bn / e.cg) * 128.0 * active / kBStreamBytesPerClk;
+                if (lat > kbc) kbc = lat;
+                if (bw > kbc) kbc = bw;
+            }
+            double unit = kb_unit * kbc + bubble;
+            if (splits > 1) unit += (e.bn / 32.0) * ((splits + 1) / 2) * kL2LatencyClk + kSplitFixedClocks;
+            double cost = static_cast<double>(waves) * unit;
+            if (cost < hbm_floor) cost = hbm_floor;
+            const bool better =
+                cost < best_cost * 0.999 ||
+                (cost <= best_cost * 1.001 && best.entry &&
+                 (splits < best.splits ||
+                  (splits == best.splits && (e.cg > best.entry->cg || (e.cg == best.entry->cg && e.bn > best.entry->bn)))));
+            if (best.entry == nullptr || better) {
+                best_cost = cost;
+                best = TileChoice{&e, units, splits};
+            }
         }
     }
     return best;
@@ -245,9 +325,9 @@ dg_status check_common(const void* a, const int32_t* sfa, const void* b, const i
 }
 
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
-                      void* stream, DeviceState* st, const void* a, const void* b, int a_rank, int b_rank,
-                      uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
-    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k / 128, m_blocks_for_heuristic);
+                      long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
+                      int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
+    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes);
     const KernelEntry* e = choice.entry;
     if (e == nullptr) return DG_ERR_UNSUPPORTED;
     const int bn = e->bn;
@@ -261,13 +341,17 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     p.raster_group = 16 / cg;
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.test_mode = g_test_mode.load();
-    p.k_rotate = g_k_rotate;
+    p.splits = choice.splits;
+    p.ws = choice.splits > 1 ? st->split_ws : nullptr;
+    p.counters = choice.splits > 1 ? st->split_counters : nullptr;
+    p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
     if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
     if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats,
                           static_cast<uint32_t>(bn / cg)))
         return DG_ERR_INVALID_ARG;
     if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
-    const long long tiles = (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks);
+    const long long tiles =
+        (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks) * choice.splits;
     if (tiles <= 0) return DG_OK;
     const int units = static_cast<int>(tiles < choice.units ? tiles : choice.units);
     void* args[] = {&p};
@@ -284,8 +368,9 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     cfg.attrs = attr;
     cfg.numAttrs = cg == 2 ? 1 : 0;
     if (g_log)
-        std::fprintf(stderr, "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d grid=%d (units %d) smem=%d\n",
-                     kind, p.rows, p.n, p.k, p.groups, bn, cg, units * cg, choice.units, e->smem);
+        std::fprintf(stderr,
+                     "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d splits=%d grid=%d (units %d) smem=%d\n",
+                     kind, p.rows, p.n, p.k, p.groups, bn, cg, choice.splits, units * cg, choice.units, e->smem);
     cudaError_t err = cudaLaunchKernelExC(&cfg, e->fn, args);
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
@@ -319,6 +404,10 @@ dg_status dgb200_device_error(uint32_t* bits, int clear) {
     if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
     if (cudaMemcpy(bits, st->status, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
     if (clear && cudaMemset(st->status, 0, sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+    // a launch that gave up may have left split-K counters part-way
+    if (clear && *bits != 0 && st->split_counters != nullptr &&
+        cudaMemset(st->split_counters, 0, kSplitCounters * sizeof(uint32_t)) != cudaSuccess)
+        return DG_ERR_CUDA;
     return DG_OK;
 }
 
@@ -337,6 +426,12 @@ dg_status dgb200_set_block_n(int block_n) {
 dg_status dgb200_set_cta_group(int cta_group) {
     if (cta_group < 0 || cta_group > 2) return DG_ERR_UNSUPPORTED;
     g_force_cg.store(cta_group);
+    return DG_OK;
+}
+
+dg_status dgb200_set_splits(int splits) {
+    if (splits < 0 || splits > kMaxSplits) return DG_ERR_UNSUPPORTED;
+    g_force_splits.store(splits);
     return DG_OK;
 }
 
@@ -366,7 +461,8 @@ dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const in
     p.k = K;
     p.groups = 1;
     p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
-    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, stream, st, a, b, 2, 2,
+    const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
+    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
                        static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
 }
 
@@ -390,7 +486,9 @@ dg_status m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, co
     p.k = K;
     p.groups = G;
     p.num_m_blocks = (M_total + dg::BM - 1) / dg::BM;
-    return launch_gemm(dg::kContiguous, p, p.num_m_blocks, p.num_m_blocks, stream, st, a, b, 2, 3,
+    const long long bytes = static_cast<long long>(M_total) * K + static_cast<long long>(G) * N * K +
+                            2LL * M_total * N;
+    return launch_gemm(dg::kContiguous, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 3,
                        static_cast<uint64_t>(M_total), 1, static_cast<uint64_t>(N), static_cast<uint64_t>(G));
 }
 
@@ -415,7 +513,8 @@ dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const 
     p.groups = G;
     p.num_m_blocks = (max_m + dg::BM - 1) / dg::BM;
     const long long mb_total = static_cast<long long>(G) * p.num_m_blocks;
-    return launch_gemm(dg::kMasked, p, mb_total, mb_total, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
+    const long long bytes = static_cast<long long>(G) * N * K;  // the weights; the valid rows are unknown here
+    return launch_gemm(dg::kMasked, p, mb_total, mb_total, bytes, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
                        static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
 }
 

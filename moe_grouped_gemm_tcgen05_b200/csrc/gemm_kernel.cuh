@@ -102,6 +102,12 @@ struct GemmParams {
     uint64_t wait_limit_ns;   // bound of every mbarrier wait
     int k_rotate;             // 1: each tile walks its K groups starting at group (tile mod groups)
     int test_mode;            // 1: CTA 0 withholds its first scale-group arrive (exercises the timeout path)
+    // split-K (dense form, single CTAs): each output tile is computed by `splits`
+    // work units over disjoint ranges of K groups; the last one to finish adds
+    // the fp32 partials in split order and writes the bf16 tile
+    int splits;               // 1 = no split; range i covers K groups [i*G/splits, (i+1)*G/splits)
+    float* ws;                // partials: [tile][split][4 row quarters][BN/4][32 lanes][4]
+    uint32_t* counters;       // finished units per output tile; zero between calls
 };
 
 template <int BN, int CG, bool SCHED_SMEM>
@@ -142,6 +148,8 @@ struct GemmConfig {
 
 struct Tile {
     int m_blk, n_blk, g;      // g: group (masked) or expert (contiguous), 0 for dense
+    int kg0, kg1;             // K groups [kg0, kg1) of this work unit
+    int base, split;          // output tile index and split index (split-K; else base = t, split = 0)
 };
 
 // ----------------------------------------------------------------- waits ----
@@ -193,9 +201,16 @@ __device__ __forceinline__ void sleep_ns(uint64_t ns) {
 // Dense / contiguous: banded raster. Within a band of `raster_group` m-tiles
 // the m-tile varies fastest, so CTAs running at the same time share the B tile
 // and a bounded slab of A.
-__device__ __forceinline__ bool raster_tile(const GemmParams& p, int t, Tile& c) {
+__device__ __forceinline__ bool raster_tile(const GemmParams& p, int t_unit, Tile& c) {
+    const int t = t_unit / p.splits;          // output tile; its splits are consecutive work units
+    const int split = t_unit - t * p.splits;
     const int total = p.num_m_blocks * p.num_n_blocks;
     if (t >= total) return false;
+    c.base = t;
+    c.split = split;
+    const int kgc = (p.kb + 3) / 4;  // K groups of four 128-K blocks
+    c.kg0 = split * kgc / p.splits;
+    c.kg1 = (split + 1) * kgc / p.splits;
     const int band_tiles = p.raster_group * p.num_n_blocks;
     const int band = t / band_tiles;
     const int local = t - band * band_tiles;
@@ -218,6 +233,8 @@ __device__ __forceinline__ bool masked_tile(const int* s_prefix, const int* s_mm
     c.g = gcur;
     c.n_blk = local / mb;
     c.m_blk = local - c.n_blk * mb;
+    c.base = t;
+    c.split = 0;
     return true;
 }
 
@@ -240,6 +257,8 @@ template <int KIND, bool NEED_EXPERT>
 __device__ __forceinline__ bool next_tile(const GemmParams& p, const int* s_prefix, const int* s_mm, int t,
                                           int& gcur, Tile& c, uint32_t lane) {
     if constexpr (KIND == kMasked) {
+        c.kg0 = 0;
+        c.kg1 = (p.kb + 3) / 4;
         return masked_tile(s_prefix, s_mm, p.groups, t, gcur, c);
     } else {
         if (!raster_tile(p, t, c)) return false;
@@ -340,8 +359,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     uint64_t* tfull_bar = sf_empty_bar + SF_RING;    // accumulator ready for the epilogue
     uint64_t* tempty_bar = tfull_bar + 2;            // accumulator drained by the epilogue(s)
     uint64_t* drain_bar = tempty_bar + 2;            // all MMAs issued for this CTA finished
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(drain_bar + 1);
+    uint64_t* epi_bar = drain_bar + 1;               // split-K: the four epilogue warps meet
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
+    volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);  // split-K: this unit reduces
     int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked)
     int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups]     (masked)
 
@@ -366,6 +387,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             mbar_init(&tempty_bar[i], 4 * CG);    // every epilogue warp of the unit
         }
         mbar_init(drain_bar, 1);
+        mbar_init(epi_bar, 4);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -429,7 +451,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             const int a_row = cur.m_blk * BM * CG + my_rows;
             const int b_row = cur.n_blk * BN + Cfg::B_ROWS * static_cast<int>(rank);
             const int g = max(cur.g, 0);
-            for (int gi = 0; gi < kg_count && !aborted; ++gi) {
+            for (int gi = cur.kg0; gi < cur.kg1 && !aborted; ++gi) {
             const int kgrp = rot_group(p, t, gi, kg_count);
             for (int kb = 4 * kgrp; kb < min(4 * kgrp + 4, p.kb); ++kb) {
                 if (!wait_warp(&empty_bar[stage], phase ^ 1u, p, s_abort)) { aborted = true; break; }
@@ -488,16 +510,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // Groups are visited in the MMA warp's order (tile by tile, K groups
             // in order). Two register sets keep the loads of two groups in
             // flight while a third is stored.
-            int ct = unit, ckg = 0, cg_cur = 0;
+            int ct = unit, cg_cur = 0;
             Tile ctile;
             bool cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+            int ckg = cok ? ctile.kg0 : 0;
             auto load_next = [&](ScaleWords<BN, KIND, CG>& w) -> bool {
                 if (!cok) return false;
                 w.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, rot_group(p, ct, ckg, kg_count), lane);
-                if (++ckg == kg_count) {
-                    ckg = 0;
+                if (++ckg == ctile.kg1) {
                     ct += units;
                     cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+                    if (cok) ckg = ctile.kg0;
                 }
                 return true;
             };
@@ -560,7 +583,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 if (!wait_warp(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
                 tc_fence_after();  // the epilogue's TMEM reads precede the MMAs below
                 const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
-                for (int gi = 0; gi < kg_count && !aborted; ++gi) {
+                for (int gi = c.kg0; gi < c.kg1 && !aborted; ++gi) {
                     const int kgrp = rot_group(p, t, gi, kg_count);
                     // this group's scale words (both CTAs of a pair) -> TMEM; the
                     // slot is free again once the copy has completed
@@ -596,7 +619,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                                 // advance the start address by 32 bytes of K inside the swizzled row
                                 const uint64_t koff = static_cast<uint64_t>((k * MMA_K) >> 4);
                                 tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
-                                                                sfb_t, (gi > 0 || kb > 4 * kgrp || k > 0) ? 1u : 0u);
+                                                                sfb_t, (gi > c.kg0 || kb > 4 * kgrp || k > 0) ? 1u : 0u);
                             }
                             tc_commit<CG>(&empty_bar[stage]);
                         }
@@ -627,6 +650,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         if constexpr (CG == 2) tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
         int acc = 0;
         uint32_t acc_phase = 0;
+        uint32_t epi_phase = 0;
         int gcur = 0;
         int buf = 0;
         Tile c;
@@ -656,62 +680,160 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_COLS;
             const int n0 = c.n_blk * BN;
             __nv_bfloat16* drow = p.d + out_row * static_cast<size_t>(p.n) + n0;
+            constexpr int kMaxBatch = 128;
+            // split-K (dense, single CTAs): every unit parks its fp32 partial
+            // in the workspace; the unit that finishes a tile last adds the
+            // partials in split order (the same sum whichever unit is last)
+            // and writes the bf16 tile.
+            constexpr bool kCanSplit = KIND == kDense && CG == 1;
+            const bool split = kCanSplit && p.splits > 1;
+            bool emit_tile = !split;
+            if constexpr (kCanSplit) {
+                if (split) {
+                    float* part = p.ws + ((static_cast<size_t>(c.base) * p.splits + c.split) * 4 + q) * (BN * 32);
 #pragma unroll
-            for (int h = 0; h < BN; h += 128) {
-                constexpr int kMaxBatch = 128;
-                const int cols = (BN - h) < kMaxBatch ? (BN - h) : kMaxBatch;  // compile-time after unrolling
-                uint32_t r[kMaxBatch];
+                    for (int h = 0; h < BN; h += 128) {
+                        const int cols = (BN - h) < kMaxBatch ? (BN - h) : kMaxBatch;
+                        uint32_t r[kMaxBatch];
 #pragma unroll
-                for (int j = 0; j < kMaxBatch / 32; ++j)
-                    if (32 * j < cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
-                tc_wait_ld();
-                if (h + 128 >= BN) {
-                    // last TMEM read of this accumulator: hand it back to the MMA warp
-                    tc_fence_before();
+                        for (int j = 0; j < kMaxBatch / 32; ++j)
+                            if (32 * j < cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
+                        tc_wait_ld();
+                        if (h + 128 >= BN) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int c4 = 0; c4 < kMaxBatch / 4; ++c4)
+                                if (4 * c4 < cols)
+                                    __stcg(reinterpret_cast<float4*>(part + ((h / 4 + c4) * 32 + lane) * 4),
+                                           make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
+                                                       __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3])));
+                        }
+                    }
+                    // publish: every thread's partial stores precede the count
+                    __threadfence();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(epi_bar);
+                    if (!wait_warp(epi_bar, epi_phase, p, s_abort)) break;
+                    epi_phase ^= 1u;
+                    if (warp == 2 && lane == 0) {
+                        const uint32_t done = atomicAdd(&p.counters[c.base], 1u);
+                        const bool last = done == static_cast<uint32_t>(p.splits - 1);
+                        if (last) atomicExch(&p.counters[c.base], 0u);  // zero again for the next call
+                        *s_last = last ? 1 : 0;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(epi_bar);
+                    if (!wait_warp(epi_bar, epi_phase, p, s_abort)) break;
+                    epi_phase ^= 1u;
+                    emit_tile = *s_last != 0;
+                    if (emit_tile) __threadfence();  // the other units' partials are visible from here on
+                }
+            }
+            // fp32 -> bf16 (round to nearest even) of 32 columns starting at tile
+            // column hc, written as one 32x32 chunk
+            auto emit32 = [&](const uint32_t* v, int hc) {
+                const int col = n0 + hc;
+                if (col >= p.n) return;  // warp-uniform: N tail
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    w[i] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+                if (use_tma) {
+                    // the store issued two chunks ago has finished reading this buffer
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    uint8_t* sb = stg + buf * 2048;
+                    // 32 rows x 64 bytes with the 64-byte swizzle: granule g of
+                    // row r sits at granule g ^ ((r >> 1) & 3)
+                    const uint32_t sw = (lane >> 1) & 3u;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
+                            make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+                    fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
-                        if (CG == 1 || leader) mbar_arrive(&tempty_bar[acc]);
-                        else mbar_arrive_cluster(tempty_leader0 + 8u * static_cast<uint32_t>(acc));
+                        if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
+                        else tma_store_2d(&p.tma_d, sb, col, row_coord);
+                        bulk_commit_group();
                     }
+                    buf ^= 1;
+                } else if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        if (col + 8 * q4 < p.n)
+                            *reinterpret_cast<uint4*>(drow + hc + 8 * q4) =
+                                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
                 }
+            };
+            if (emit_tile && !(kCanSplit && split)) {
 #pragma unroll
-                for (int j = 0; j < kMaxBatch / 32; ++j) {
-                    if (32 * j >= cols) continue;
-                    const int col = n0 + h + 32 * j;
-                    if (col >= p.n) continue;  // warp-uniform: N tail
-                    uint32_t w[16];
+                for (int h = 0; h < BN; h += 128) {
+                    const int cols = (BN - h) < kMaxBatch ? (BN - h) : kMaxBatch;  // compile-time after unrolling
+                    uint32_t r[kMaxBatch];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[32 * j + 2 * i]),
-                                                                  __uint_as_float(r[32 * j + 2 * i + 1]));
-                        w[i] = *reinterpret_cast<uint32_t*>(&b2);
-                    }
-                    if (use_tma) {
-                        // the store issued two chunks ago has finished reading this buffer
-                        if (lane == 0) bulk_wait_group_read<1>();
-                        __syncwarp();
-                        uint8_t* sb = stg + buf * 2048;
-                        // 32 rows x 64 bytes with the 64-byte swizzle: granule g of
-                        // row r sits at granule g ^ ((r >> 1) & 3)
-                        const uint32_t sw = (lane >> 1) & 3u;
-#pragma unroll
-                        for (int g = 0; g < 4; ++g)
-                            *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
-                                make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-                        fence_proxy_async_smem();
+                    for (int j = 0; j < kMaxBatch / 32; ++j)
+                        if (32 * j < cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
+                    tc_wait_ld();
+                    if (h + 128 >= BN) {
+                        // last TMEM read of this accumulator: hand it back to the MMA warp
+                        tc_fence_before();
                         __syncwarp();
                         if (lane == 0) {
-                            if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
-                            else tma_store_2d(&p.tma_d, sb, col, row_coord);
-                            bulk_commit_group();
+                            if (CG == 1 || leader) mbar_arrive(&tempty_bar[acc]);
+                            else mbar_arrive_cluster(tempty_leader0 + 8u * static_cast<uint32_t>(acc));
                         }
-                        buf ^= 1;
-                    } else if (valid) {
+                    }
 #pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            if (col + 8 * v < p.n)
-                                *reinterpret_cast<uint4*>(drow + h + 32 * j + 8 * v) =
-                                    make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                    for (int j = 0; j < kMaxBatch / 32; ++j)
+                        if (32 * j < cols) emit32(r + 32 * j, h + 32 * j);
+                }
+            }
+            if constexpr (kCanSplit) {
+                if (emit_tile && split) {
+                    // this unit finished the tile last: the sum of the partials in
+                    // split order, 32 columns at a time, loads of two splits in
+                    // flight per round
+                    const float* tile_ws = p.ws + (static_cast<size_t>(c.base) * p.splits * 4 + q) * (BN * 32);
+                    const size_t split_stride = static_cast<size_t>(4) * BN * 32;
+#pragma unroll 1
+                    for (int hc = 0; hc < BN; hc += 32) {
+                        float acc32[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc32[i] = 0.f;
+                        if (valid) {
+                            const float* src = tile_ws + ((hc / 4) * 32 + lane) * 4;
+                            for (int sp0 = 0; sp0 < p.splits; sp0 += 2) {
+                                float4 v[2][8];
+#pragma unroll
+                                for (int u = 0; u < 2; ++u)
+                                    if (sp0 + u < p.splits)
+#pragma unroll
+                                        for (int c4 = 0; c4 < 8; ++c4)
+                                            v[u][c4] = __ldcg(reinterpret_cast<const float4*>(
+                                                src + (sp0 + u) * split_stride + c4 * 128));
+#pragma unroll
+                                for (int u = 0; u < 2; ++u)
+                                    if (sp0 + u < p.splits)
+#pragma unroll
+                                        for (int c4 = 0; c4 < 8; ++c4) {
+                                            acc32[4 * c4] += v[u][c4].x;
+                                            acc32[4 * c4 + 1] += v[u][c4].y;
+                                            acc32[4 * c4 + 2] += v[u][c4].z;
+                                            acc32[4 * c4 + 3] += v[u][c4].w;
+                                        }
+                            }
+                        }
+                        uint32_t bits[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) bits[i] = __float_as_uint(acc32[i]);
+                        emit32(bits, hc);
                     }
                 }
             }

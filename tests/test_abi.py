@@ -76,3 +76,19 @@ def test_binding_fails_loudly_without_cuda():
     with pytest.raises(ValueError):
         dg.fp8_gemm_nt(a, torch.zeros((128, 1), dtype=torch.int32), a,
                        torch.zeros((1, 1), dtype=torch.int32), torch.zeros((128, 128), dtype=torch.bfloat16))
+
+
+def test_tuning_switch_ranges(lib):
+    """The process-wide tuning switches reject values outside their ranges and
+    need no device to do so (0 restores the heuristic in each)."""
+    for name, good, bad in (("dgb200_set_block_n", (0, 64, 224, 256), (-1, 100, 512)),
+                            ("dgb200_set_cta_group", (0, 1, 2), (-1, 3)),
+                            ("dgb200_set_splits", (0, 1, 2, 16), (-1, 17))):
+        f = getattr(lib, name)
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.c_int]
+        for v in good:
+            assert f(v) == 0, (name, v)
+        for v in bad:
+            assert f(v) == 3, (name, v)   # DG_ERR_UNSUPPORTED
+        assert f(0) == 0

@@ -61,3 +61,28 @@ def test_timeout_is_reported_and_context_survives(form):
     check_fp(bf16_to_f64(dm)[valid], refm[valid], "masked after timeout")
     assert dg.device_error(clear=True) == 0
     dg.set_cta_group(0)
+
+
+def test_timeout_under_split_k_then_counters_are_zeroed():
+    """A split-K launch that gives up leaves per-tile counters part-way;
+    clearing the status word zeroes them, so the next split-K calls are right."""
+    dg.init()
+    dg.device_error(clear=True)
+    dg.set_splits(4)
+    p = W.dense(200, 512, 4096, seed=33)
+    try:
+        dg.set_test_hooks(1, 200)
+        _dense(p)
+        torch.cuda.synchronize()
+        assert dg.device_error(clear=True) & dg.DEVERR_TIMEOUT
+    finally:
+        dg.set_test_hooks(0, 0)
+    ref = oracle.fp8_gemm_nt(p["a"], oracle.pack_ue8m0(p["sfa_f32"]), p["b"], oracle.pack_ue8m0(p["sfb_f32"]))
+    try:
+        for _ in range(3):
+            d = _dense(p)
+            torch.cuda.synchronize()
+            check_fp(bf16_to_f64(d), ref, "split-K after timeout")
+        assert dg.device_error(clear=True) == 0
+    finally:
+        dg.set_splits(0)
