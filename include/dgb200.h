@@ -71,7 +71,9 @@ typedef enum {
     DG_ERR_ALIGNMENT = 2,      /* pointer or row pitch not aligned as required */
     DG_ERR_UNSUPPORTED = 3,    /* valid request outside this build's limits */
     DG_ERR_NOT_INITIALIZED = 4,/* no usable CUDA device / driver entry point */
-    DG_ERR_CUDA = 5            /* a CUDA runtime call or launch failed */
+    DG_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+    DG_ERR_SCRATCH_TOO_SMALL = 6 /* fp8_gemm_nt_noalloc: the request needs more
+                                    scratch than its static arrays hold */
 } dg_status;
 
 /* Bits of the device status word (see dgb200_device_error). */
@@ -154,6 +156,36 @@ DG_API dg_status dgb200_set_test_hooks(int mode, int wait_limit_ms);
  */
 DG_API dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
                       void* d, int M, int N, int K, void* stream);
+
+/*
+ * fp8_gemm_nt_noalloc: the dense GEMM of fp8_gemm_nt (same arguments, layouts,
+ * limits and results) that allocates no device memory, on any call. The pages
+ * of the method have no counterpart of this call; it exists for callers that
+ * may not allocate (a framework whose caching allocator already holds the
+ * device's memory, a server that plans all memory up front and forbids
+ * allocation on the request path, code that must not let cudaMalloc/cudaFree
+ * synchronise the device).
+ *   splits : 0 = the tile model's choice among configurations whose split-K
+ *            scratch fits the static arrays below (never DG_ERR_SCRATCH_TOO_SMALL);
+ *            1 = no split-K; s >= 2 = exactly s ranges of K groups, tiled as
+ *            fp8_gemm_nt with dgb200_set_splits(s) would tile them.
+ * Split-K scratch lives in file-scope __device__ arrays of the library, found
+ * with cudaGetSymbolAddress: at most 8 MiB of fp32 partials (2^21 floats; a
+ * split call needs ceil(M/128) * ceil(N/BN) * s * 128 * BN * 4 bytes for its N
+ * tile BN) and 1024 output tiles. A request beyond either limit returns
+ * DG_ERR_SCRATCH_TOO_SMALL before any device work; s > 16 returns
+ * DG_ERR_UNSUPPORTED. A splitting call first zeroes the tile counters it uses
+ * (an asynchronous memset on `stream`).
+ * The scratch is shared by every caller of this function on a device: calls
+ * that overlap in time (two streams, two host threads, or one call still
+ * running when the next one starts on another stream) race on it and give
+ * wrong results. Calls on one stream are ordered and safe.
+ * The first call on a device does per-device set-up (kernel attributes,
+ * symbol addresses; no allocation) and should come before any stream capture
+ * that includes this call.
+ */
+DG_API dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                                     int M, int N, int K, int splits, void* stream);
 
 /*
  * Contiguous M-grouped FP8 GEMM for MoE ("DeepGEMM tested by Novita AI",

@@ -24,6 +24,7 @@ __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
+    "fp8_gemm_nt_noalloc",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -38,7 +39,7 @@ _lock = threading.Lock()
 
 _STATUS = {
     0: "DG_OK", 1: "DG_ERR_INVALID_ARG", 2: "DG_ERR_ALIGNMENT", 3: "DG_ERR_UNSUPPORTED",
-    4: "DG_ERR_NOT_INITIALIZED", 5: "DG_ERR_CUDA",
+    4: "DG_ERR_NOT_INITIALIZED", 5: "DG_ERR_CUDA", 6: "DG_ERR_SCRATCH_TOO_SMALL",
 }
 
 
@@ -84,6 +85,8 @@ def load():
         L.dgb200_set_test_hooks.argtypes = [i32, i32]
         L.fp8_gemm_nt.restype = i32
         L.fp8_gemm_nt.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
+        L.fp8_gemm_nt_noalloc.restype = i32
+        L.fp8_gemm_nt_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_contiguous.restype = i32
         L.m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_masked.restype = i32
@@ -180,6 +183,24 @@ def fp8_gemm_nt(a, sfa, b, sfb, d):
     _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
     _need(d, "d", _BF16, (M, N))
     _check("fp8_gemm_nt", load().fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def fp8_gemm_nt_noalloc(a, sfa, b, sfb, d, splits: int = 0):
+    """fp8_gemm_nt that allocates no device memory: split-K scratch comes from
+    static arrays of the library (8 MiB of partials, 1024 tiles). splits: 0 =
+    model's choice within that scratch, 1 = none, s >= 2 = exactly s. Calls that
+    overlap in time on one device race on the scratch (see include/dgb200.h)."""
+    _need(a, "a", _FP8)
+    M, K = a.shape
+    _need(b, "b", _FP8)
+    N = b.shape[0]
+    _need(b, "b", _FP8, (N, K))
+    _need(sfa, "sfa", _I32, (M, _kp(K)))
+    _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (M, N))
+    _check("fp8_gemm_nt_noalloc", load().fp8_gemm_nt_noalloc(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K,
+                                                             int(splits), _stream()))
     return d
 
 

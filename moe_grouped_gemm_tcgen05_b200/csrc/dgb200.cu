@@ -25,6 +25,20 @@
 // Device status word (DG_DEVERR_* bits). One per device that loads the library.
 __device__ uint32_t g_dg_device_status = 0;
 
+// Split-K scratch of fp8_gemm_nt_noalloc, part of the module image instead of
+// an allocation. Some callers may not allocate device memory at all: a
+// framework whose caching allocator has already reserved the device's memory
+// (a library cudaMalloc then fails, or fragments the pool behind its back), a
+// server that plans every byte up front and treats an allocation on the
+// request path as a latency spike and an out-of-memory risk, or code running
+// where cudaMalloc / cudaFree would synchronise the device at a bad moment.
+// These arrays exist as soon as the module is loaded; calls find them with
+// cudaGetSymbolAddress. Limits: 8 MiB of fp32 partials, 1024 output tiles.
+constexpr size_t kStaticPartialFloats = size_t(2) << 20;
+constexpr int kStaticCounters = 1024;
+static __device__ __align__(256) float g_noalloc_partials[kStaticPartialFloats];
+static __device__ __align__(256) uint32_t g_noalloc_counters[kStaticCounters];
+
 namespace {
 
 using dg::GemmParams;
@@ -47,6 +61,9 @@ struct DeviceState {
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
+// Per-device state of fp8_gemm_nt_noalloc: the same set-up without the
+// workspace allocation; split_ws / split_counters point at the static arrays.
+DeviceState g_dev_noalloc[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_bn{0};
 std::atomic<int> g_force_cg{0};
@@ -96,11 +113,10 @@ constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
 
 // ------------------------------------------------------------------ init ----
 
-dg_status init_device(int dev) {
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
-    DeviceState& st = g_dev[dev];
-    if (st.ready) return DG_OK;
+// Per-device set-up that allocates no device memory: the driver's tensor-map
+// encoder, the architecture check, SM count, kernel attributes, co-resident
+// CTA pairs and the address of the status word. Caller holds g_mu.
+dg_status setup_device(int dev, DeviceState& st) {
     if (g_encode == nullptr) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -141,6 +157,16 @@ dg_status init_device(int dev) {
     void* status = nullptr;
     if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
     st.status = static_cast<uint32_t*>(status);
+    return DG_OK;
+}
+
+dg_status init_device(int dev) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    DeviceState& st = g_dev[dev];
+    if (st.ready) return DG_OK;
+    const dg_status s = setup_device(dev, st);
+    if (s != DG_OK) return s;
     // split-K workspace: optional; without it the GEMMs run unsplit
     void* ws = nullptr;
     void* ctr = nullptr;
@@ -155,6 +181,28 @@ dg_status init_device(int dev) {
         cudaGetLastError();  // clear the allocation error; split-K stays off
     }
     st.ready = true;
+    return DG_OK;
+}
+
+dg_status noalloc_device(DeviceState** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev_noalloc[dev];
+    if (!st.ready) {
+        const dg_status s = setup_device(dev, st);
+        if (s != DG_OK) return s;
+        void* partials = nullptr;
+        void* counters = nullptr;
+        if (cudaGetSymbolAddress(&partials, g_noalloc_partials) != cudaSuccess ||
+            cudaGetSymbolAddress(&counters, g_noalloc_counters) != cudaSuccess)
+            return DG_ERR_CUDA;
+        st.split_ws = static_cast<float*>(partials);
+        st.split_counters = static_cast<uint32_t*>(counters);
+        st.ready = true;
+    }
+    *out = &st;
     return DG_OK;
 }
 
@@ -248,13 +296,20 @@ struct TileChoice {
 // unique bytes at the HBM rate. Split-K is considered only when the output
 // tiles alone leave SMs idle; a split unit also pays for writing its fp32
 // partial and, on average, for one reduction read of all partials.
-TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                       long long unique_bytes) {
+// Split-K scratch a choice may use: partial floats and per-tile counters
+// (split_ok false: no scratch at all).
+struct SplitScratch {
+    bool split_ok;
+    double bytes;
+    long long counters;
+};
+
+TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
+                          long long unique_bytes, int forced_splits, const SplitScratch& scratch) {
     const int kb = k / 128;
     const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
     const int forced_cg = kind == dg::kDense ? g_force_cg.load() : 0;  // pairs exist for the dense form only
-    const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
     TileChoice best{nullptr, 0, 1};
     double best_cost = 1e300;
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
@@ -274,12 +329,12 @@ TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, 
         const double bubble = num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0;
         for (int splits = 1; splits <= kMaxSplits; ++splits) {
             if (forced_splits != 0 && splits != forced_splits) continue;
-            const bool can_split = kind == dg::kDense && e.cg == 1 && st->split_ws != nullptr;
+            const bool can_split = kind == dg::kDense && e.cg == 1 && scratch.split_ok;
             if (splits > 1) {
                 if (!can_split || splits > kg) break;
                 if (forced_splits == 0 && tiles >= units) break;  // the tiles alone fill the GPU
-                if (tiles > kSplitCounters) break;
-                if (static_cast<double>(tiles) * splits * dg::BM * e.bn * sizeof(float) > kSplitWsBytes) break;
+                if (tiles > scratch.counters) break;
+                if (static_cast<double>(tiles) * splits * dg::BM * e.bn * sizeof(float) > scratch.bytes) break;
             }
             const int gps = (kg + splits - 1) / splits;  // K groups of the longest range
             const long long work = tiles * splits;
@@ -311,6 +366,22 @@ TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, 
     return best;
 }
 
+// The library's own choice: the allocated split-K workspace, and the split
+// count forced by dgb200_set_splits (dense form).
+TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
+                       long long unique_bytes) {
+    const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
+    const SplitScratch scratch{st->split_ws != nullptr, static_cast<double>(kSplitWsBytes), kSplitCounters};
+    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch);
+}
+
+// Bytes of split-K partials a choice writes (0 when it does not split).
+double split_bytes(const TileChoice& c, long long m128_blocks, int n) {
+    if (c.splits <= 1 || c.entry == nullptr) return 0.0;
+    const long long tiles = m128_blocks * ((n + c.entry->bn - 1) / c.entry->bn);
+    return static_cast<double>(tiles) * c.splits * dg::BM * c.entry->bn * sizeof(float);
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 dg_status check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* d, int N,
@@ -324,10 +395,12 @@ dg_status check_common(const void* a, const int32_t* sfa, const void* b, const i
     return DG_OK;
 }
 
-dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
-                      long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
-                      int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
-    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes);
+// Launch one GEMM with a given tile choice; split-K partials and counters
+// come from `ws` / `counters` (used only when the choice splits).
+dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counters, int kind, GemmParams& p,
+                           long long max_tiles_per_nblock, void* stream, const DeviceState* st, const void* a,
+                           const void* b, int a_rank, int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows,
+                           uint64_t b_mats) {
     const KernelEntry* e = choice.entry;
     if (e == nullptr) return DG_ERR_UNSUPPORTED;
     const int bn = e->bn;
@@ -342,8 +415,8 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.test_mode = g_test_mode.load();
     p.splits = choice.splits;
-    p.ws = choice.splits > 1 ? st->split_ws : nullptr;
-    p.counters = choice.splits > 1 ? st->split_counters : nullptr;
+    p.ws = choice.splits > 1 ? ws : nullptr;
+    p.counters = choice.splits > 1 ? counters : nullptr;
     p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
     if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
     if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats,
@@ -375,6 +448,14 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
+dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
+                      long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
+                      int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
+    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes);
+    return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
+                            a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
+}
+
 }  // namespace
 
 extern "C" {
@@ -387,6 +468,7 @@ const char* dgb200_status_string(dg_status s) {
         case DG_ERR_UNSUPPORTED: return "DG_ERR_UNSUPPORTED";
         case DG_ERR_NOT_INITIALIZED: return "DG_ERR_NOT_INITIALIZED";
         case DG_ERR_CUDA: return "DG_ERR_CUDA";
+        case DG_ERR_SCRATCH_TOO_SMALL: return "DG_ERR_SCRATCH_TOO_SMALL";
     }
     return "DG_ERR_UNKNOWN";
 }
@@ -464,6 +546,56 @@ dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const in
     const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
     return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
                        static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+}
+
+dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                              int N, int K, int splits, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M <= 0) return DG_ERR_INVALID_ARG;
+    if (splits < 0 || splits > kMaxSplits) return DG_ERR_UNSUPPORTED;
+    DeviceState* st = nullptr;
+    if ((s = noalloc_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = nullptr;
+    p.rows = M;
+    p.n = N;
+    p.k = K;
+    p.groups = 1;
+    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
+    const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
+    const double static_bytes = static_cast<double>(kStaticPartialFloats) * sizeof(float);
+    TileChoice choice;
+    if (splits == 0) {
+        // the model's choice among what fits the static scratch
+        const SplitScratch scratch{true, static_bytes, kStaticCounters};
+        choice = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, 0, scratch);
+    } else {
+        // exactly `splits` ranges, tiled as the model would with unlimited
+        // scratch; refused if that needs more than the static arrays hold
+        const SplitScratch unlimited{true, 1e300, 1LL << 40};
+        choice = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, splits, unlimited);
+        if (choice.entry == nullptr) return DG_ERR_UNSUPPORTED;
+        if (choice.splits > 1) {
+            const long long tiles = p.num_m_blocks * ((N + choice.entry->bn - 1) / choice.entry->bn);
+            if (split_bytes(choice, p.num_m_blocks, N) > static_bytes || tiles > kStaticCounters)
+                return DG_ERR_SCRATCH_TOO_SMALL;
+        }
+    }
+    if (choice.entry == nullptr) return DG_ERR_UNSUPPORTED;
+    if (choice.splits > 1) {
+        // the counters must start at zero (a launch that gave up may have left some part-way)
+        const long long tiles = p.num_m_blocks * ((N + choice.entry->bn - 1) / choice.entry->bn);
+        if (cudaMemsetAsync(st->split_counters, 0, static_cast<size_t>(tiles) * sizeof(uint32_t),
+                            static_cast<cudaStream_t>(stream)) != cudaSuccess)
+            return DG_ERR_CUDA;
+    }
+    return launch_gemm_with(choice, st->split_ws, st->split_counters, dg::kDense, p, p.num_m_blocks, stream, st, a, b,
+                            2, 2, static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
 }
 
 dg_status m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
