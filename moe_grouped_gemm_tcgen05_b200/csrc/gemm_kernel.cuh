@@ -577,33 +577,47 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             int gcur = 0;
             Tile c;
             bool aborted = false;
-            uint32_t sf_tmem = tmem_base + Cfg::SF_BASE;
-            uint32_t sf_other = sf_tmem + Cfg::SF_COLS;
+            // Two sets of scale columns: `sf_cur` feeds the MMAs of the current
+            // group; the next group's words are copied into `sf_nxt` right after
+            // the current group's first K-block is issued, so that wait and
+            // copy overlap MMAs already queued (the tensor pipe runs a thread's
+            // copies and MMAs in issue order).
+            uint32_t sf_cur = tmem_base + Cfg::SF_BASE;
+            uint32_t sf_nxt = sf_cur + Cfg::SF_COLS;
+            // next group's scale words (both CTAs of a pair) -> TMEM at `dst`;
+            // the ring slot is free again once the copy has completed
+            auto copy_scales = [&](uint32_t dst) -> bool {
+                if (!wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort)) return false;
+                tc_fence_after();
+                if (elect_one()) {
+                    const uint8_t* sf_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
+                    tc_cp_32x128b_warpx4<CG>(dst, smem_desc_sf(smem_u32(sf_slot)));
+#pragma unroll
+                    for (int ch = 0; ch < Cfg::SFB_CHUNKS; ++ch)
+                        tc_cp_32x128b_warpx4<CG>(dst + 4 + 4 * ch,
+                                                 smem_desc_sf(smem_u32(sf_slot + Cfg::SFA_BYTES + 512 * ch)));
+                    tc_commit<CG>(&sf_empty_bar[slot]);
+                }
+                __syncwarp();
+                if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
+                return true;
+            };
             for (int t = unit; !aborted && next_tile<KIND, false>(p, s_prefix, s_mm, t, gcur, c, lane); t += units) {
                 if (!wait_warp(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
                 tc_fence_after();  // the epilogue's TMEM reads precede the MMAs below
                 const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
+                // the tile's first group: its scales go to the set the previous
+                // group did not use
+                if (!copy_scales(sf_nxt)) { aborted = true; break; }
+                {
+                    const uint32_t tmp = sf_cur;
+                    sf_cur = sf_nxt;
+                    sf_nxt = tmp;
+                }
                 for (int gi = c.kg0; gi < c.kg1 && !aborted; ++gi) {
                     const int kgrp = rot_group(p, t, gi, kg_count);
-                    // this group's scale words (both CTAs of a pair) -> TMEM; the
-                    // slot is free again once the copy has completed
-                    if (!wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort)) { aborted = true; break; }
-                    tc_fence_after();
-                    if (elect_one()) {
-                        const uint8_t* sf_slot = smem_sf + slot * Cfg::SF_SLOT_BYTES;
-                        tc_cp_32x128b_warpx4<CG>(sf_tmem, smem_desc_sf(smem_u32(sf_slot)));
-#pragma unroll
-                        for (int ch = 0; ch < Cfg::SFB_CHUNKS; ++ch)
-                            tc_cp_32x128b_warpx4<CG>(sf_tmem + 4 + 4 * ch,
-                                                     smem_desc_sf(smem_u32(sf_slot + Cfg::SFA_BYTES + 512 * ch)));
-                        tc_commit<CG>(&sf_empty_bar[slot]);
-                    }
-                    __syncwarp();
-                    if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
-                    const uint32_t sf_cur = sf_tmem;
-                    sf_tmem = sf_other;
-                    sf_other = sf_cur;
-                    for (int kb = 4 * kgrp; kb < min(4 * kgrp + 4, p.kb); ++kb) {
+                    const int kb0 = 4 * kgrp;
+                    for (int kb = kb0; kb < min(kb0 + 4, p.kb); ++kb) {
                         // TMA bytes observed complete on the barrier are visible to
                         // the tensor core's shared-memory reads: no fence needed here
                         if (!wait_warp(&full_bar[stage], phase, p, s_abort)) { aborted = true; break; }
@@ -619,12 +633,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                                 // advance the start address by 32 bytes of K inside the swizzled row
                                 const uint64_t koff = static_cast<uint64_t>((k * MMA_K) >> 4);
                                 tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
-                                                                sfb_t, (gi > c.kg0 || kb > 4 * kgrp || k > 0) ? 1u : 0u);
+                                                                sfb_t, (gi > c.kg0 || kb > kb0 || k > 0) ? 1u : 0u);
                             }
                             tc_commit<CG>(&empty_bar[stage]);
                         }
                         __syncwarp();
                         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                        if (kb == kb0 && gi + 1 < c.kg1 && !copy_scales(sf_nxt)) { aborted = true; break; }
+                    }
+                    if (gi + 1 < c.kg1) {
+                        const uint32_t tmp = sf_cur;
+                        sf_cur = sf_nxt;
+                        sf_nxt = tmp;
                     }
                 }
                 if (aborted) break;
