@@ -107,9 +107,10 @@ DG_API dg_status dgb200_set_block_n(int block_n);
 DG_API int dgb200_block_n_supported(int block_n);
 
 /*
- * Force the dense GEMM to run on single CTAs (1) or on CTA pairs (2, tcgen05
- * cta_group::2 with a 256-row tile); 0 restores the heuristic. The grouped
- * forms always use single CTAs. Process-wide; meant for tests and tuning.
+ * Force the dense and contiguous GEMMs to run on single CTAs (1) or on CTA
+ * pairs (2, tcgen05 cta_group::2 with a 256-row tile); 0 restores the
+ * heuristic. The masked form always uses single CTAs. Process-wide; meant for
+ * tests and tuning.
  * Returns DG_ERR_UNSUPPORTED for other values; a forced combination of tile
  * width and group that is not built makes the GEMM calls return
  * DG_ERR_UNSUPPORTED.

@@ -76,6 +76,7 @@ constexpr int MMA_K = 32;               // K of one kind::mxf8f6f4 MMA
 constexpr int NUM_THREADS = 224;
 constexpr int SF_RING = 4;              // scale-word groups in flight
 constexpr int MAX_MASKED_GROUPS = 1024;
+constexpr int MAX_CACHED_BLOCKS = 1024;  // contiguous: 128-row blocks whose expert is kept in shared memory
 constexpr int SMEM_LIMIT = 232448;      // 227 KB opt-in per CTA
 constexpr uint64_t DEFAULT_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 
@@ -110,7 +111,15 @@ struct GemmParams {
     uint32_t* counters;       // finished units per output tile; zero between calls
 };
 
-template <int BN, int CG, bool SCHED_SMEM>
+// SCHED_INTS: 32-bit words of shared memory for the tile scheduler (masked:
+// clamped masked_m and tile prefix sums; contiguous: expert of every 128-row
+// block; dense: none).
+template <int KIND>
+__host__ __device__ constexpr int sched_ints() {
+    return KIND == kMasked ? 2 * MAX_MASKED_GROUPS + 8 : (KIND == kContiguous ? MAX_CACHED_BLOCKS + 8 : 16);
+}
+
+template <int BN, int CG, int SCHED_INTS>
 struct GemmConfig {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 32 in [32, 256]");
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
@@ -125,7 +134,7 @@ struct GemmConfig {
     static constexpr uint32_t TX_BYTES = CG * (A_BYTES + B_BYTES);  // TMA bytes per stage, both CTAs
     static constexpr int EPI_WARP_BYTES = 2 * 2048;             // two 32x32 bf16 staging buffers per warp
     static constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;
-    static constexpr int SCHED_BYTES = SCHED_SMEM ? (2 * MAX_MASKED_GROUPS + 8) * 4 : 64;
+    static constexpr int SCHED_BYTES = SCHED_INTS * 4;
     static constexpr int FIXED_BYTES =
         1024 /*align slack*/ + EPI_BYTES + SF_RING * SF_SLOT_BYTES + 512 /*barriers*/ + SCHED_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
@@ -150,6 +159,7 @@ struct Tile {
     int m_blk, n_blk, g;      // g: group (masked) or expert (contiguous), 0 for dense
     int kg0, kg1;             // K groups [kg0, kg1) of this work unit
     int base, split;          // output tile index and split index (split-K; else base = t, split = 0)
+    int e_own[2];             // contiguous: expert of each CTA's 128-row block (-1: padding only)
 };
 
 // ----------------------------------------------------------------- waits ----
@@ -253,16 +263,53 @@ __device__ __forceinline__ int block_expert(const GemmParams& p, int m_blk, uint
     return __reduce_max_sync(0xffffffffu, best);
 }
 
-template <int KIND, bool NEED_EXPERT>
-__device__ __forceinline__ bool next_tile(const GemmParams& p, const int* s_prefix, const int* s_mm, int t,
-                                          int& gcur, Tile& c, uint32_t lane) {
+// block_expert from the shared-memory table built in the kernel's prologue
+// when the blocks fit in it (warp-uniform either way).
+__device__ __forceinline__ int cached_block_expert(const GemmParams& p, const int* s_bexp, int blk, uint32_t lane) {
+    const int nblk = (p.rows + BM - 1) / BM;
+    if (nblk <= MAX_CACHED_BLOCKS) return blk < nblk ? s_bexp[blk] : -1;
+    return block_expert(p, blk, lane);
+}
+
+// Next work unit at or after t (stepping by `units`); false when none is left.
+// Contiguous form on CTA pairs: a pair tile covers two 128-row blocks, which
+// may belong to two experts (segments are 128-row aligned). Tiles are visited
+// in two passes over (pair, n-block): pass 0 computes the pair with the first
+// block's expert (the second block's if the first is padding only); pass 1
+// exists only when the second block has another expert, and computes the pair
+// with that one. Rows of the other expert are never written in a pass. Tiles
+// of padding only are skipped. Every role of the CTA takes the same steps.
+template <int KIND, bool NEED_EXPERT, int CG>
+__device__ __forceinline__ bool next_tile(const GemmParams& p, const int* s_prefix, const int* s_mm, int& t,
+                                          int units, int& gcur, Tile& c, uint32_t lane) {
     if constexpr (KIND == kMasked) {
         c.kg0 = 0;
         c.kg1 = (p.kb + 3) / 4;
         return masked_tile(s_prefix, s_mm, p.groups, t, gcur, c);
+    } else if constexpr (KIND == kContiguous && CG == 2) {
+        const int per_pass = p.num_m_blocks * p.num_n_blocks;
+        for (; t < 2 * per_pass; t += units) {
+            const int pass = t >= per_pass ? 1 : 0;
+            raster_tile(p, t - pass * per_pass, c);
+            const int e0 = cached_block_expert(p, s_prefix, 2 * c.m_blk, lane);
+            const int e1 = cached_block_expert(p, s_prefix, 2 * c.m_blk + 1, lane);
+            c.e_own[0] = e0;
+            c.e_own[1] = e1;
+            if (pass == 0) {
+                c.g = e0 >= 0 ? e0 : e1;
+                if (c.g >= 0) return true;
+            } else if (e0 >= 0 && e1 >= 0 && e1 != e0) {
+                c.g = e1;
+                return true;
+            }
+        }
+        return false;
     } else {
         if (!raster_tile(p, t, c)) return false;
-        if constexpr (KIND == kContiguous && NEED_EXPERT) c.g = block_expert(p, c.m_blk, lane);
+        if constexpr (KIND == kContiguous && NEED_EXPERT) {
+            c.g = cached_block_expert(p, s_prefix, c.m_blk, lane);
+            c.e_own[0] = c.g;
+        }
         return true;
     }
 }
@@ -340,8 +387,8 @@ struct ScaleWords {
 
 template <int BN, int KIND, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
-    static_assert(CG == 1 || KIND == kDense, "CTA pairs are built for the dense form");
-    using Cfg = GemmConfig<BN, CG, KIND == kMasked>;
+    static_assert(CG == 1 || KIND != kMasked, "CTA pairs are built for the dense and contiguous forms");
+    using Cfg = GemmConfig<BN, CG, sched_ints<KIND>()>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int NUM_ACC = Cfg::NUM_ACC;
 
@@ -365,6 +412,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);  // split-K: this unit reduces
     int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked)
     int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups]     (masked)
+    int* s_bexp = s_prefix;                                          // [128-row blocks] (contiguous)
 
     const uint32_t warp = threadIdx.x / 32;
     const uint32_t lane = lane_id();
@@ -429,6 +477,42 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             if (lane == 31) s_prefix[p.groups] = incl;
         }
     }
+    if constexpr (KIND == kContiguous) {
+        // expert of every 128-row block = largest valid index among its rows
+        // (-1: padding only), kept in shared memory when the blocks fit
+        // Each warp takes 8 blocks per round (lane l: rows 4l..4l+3 of each,
+        // one 16-byte load when m_indices allows) and reduces each block.
+        const int nblk = (p.rows + BM - 1) / BM;
+        if (nblk <= MAX_CACHED_BLOCKS) {
+            constexpr int kWarps = NUM_THREADS / 32;
+            const bool vec = (reinterpret_cast<uintptr_t>(p.meta) & 15) == 0;
+            auto expert_or_none = [&](int id) { return (id >= 0 && id < p.groups) ? id : -1; };
+            for (int b0 = static_cast<int>(warp) * 8; b0 < nblk; b0 += kWarps * 8) {
+                int best[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    int m = -1;
+                    const int r0 = (b0 + u) * BM + 4 * static_cast<int>(lane);
+                    if (b0 + u < nblk) {
+                        if (vec && r0 + 3 < p.rows) {
+                            const int4 v = __ldg(reinterpret_cast<const int4*>(p.meta + r0));
+                            m = max(max(expert_or_none(v.x), expert_or_none(v.y)),
+                                    max(expert_or_none(v.z), expert_or_none(v.w)));
+                        } else {
+                            for (int j = 0; j < 4; ++j)
+                                if (r0 + j < p.rows) m = max(m, expert_or_none(__ldg(p.meta + r0 + j)));
+                        }
+                    }
+                    best[u] = m;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int m = __reduce_max_sync(0xffffffffu, best[u]);
+                    if (lane == 0 && b0 + u < nblk) s_bexp[b0 + u] = m;
+                }
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
@@ -447,7 +531,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         int gcur = 0;
         Tile cur;
         bool aborted = false;
-        for (int t = unit; !aborted && next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, cur, lane); t += units) {
+        for (int t = unit; !aborted && next_tile<KIND, true, CG>(p, s_prefix, s_mm, t, units, gcur, cur, lane);
+             t += units) {
             const int a_row = cur.m_blk * BM * CG + my_rows;
             const int b_row = cur.n_blk * BN + Cfg::B_ROWS * static_cast<int>(rank);
             const int g = max(cur.g, 0);
@@ -477,7 +562,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         if (leader) mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
                         const uint32_t fb = full_leader0 + 8u * static_cast<uint32_t>(stage);
                         tma_load_2d_pair(a_dst, &p.tma_a, fb, kx, a_row);
-                        tma_load_2d_pair(b_dst, &p.tma_b, fb, kx, b_row);
+                        if constexpr (KIND == kDense) {
+                            tma_load_2d_pair(b_dst, &p.tma_b, fb, kx, b_row);
+                        } else {
+                            tma_load_3d_pair(b_dst, &p.tma_b, fb, kx, b_row, g);
+                        }
                     }
                 }
                 __syncwarp();
@@ -512,14 +601,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // flight while a third is stored.
             int ct = unit, cg_cur = 0;
             Tile ctile;
-            bool cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+            bool cok = next_tile<KIND, true, CG>(p, s_prefix, s_mm, ct, units, cg_cur, ctile, lane);
             int ckg = cok ? ctile.kg0 : 0;
             auto load_next = [&](ScaleWords<BN, KIND, CG>& w) -> bool {
                 if (!cok) return false;
                 w.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, rot_group(p, ct, ckg, kg_count), lane);
                 if (++ckg == ctile.kg1) {
                     ct += units;
-                    cok = next_tile<KIND, true>(p, s_prefix, s_mm, ct, cg_cur, ctile, lane);
+                    cok = next_tile<KIND, true, CG>(p, s_prefix, s_mm, ct, units, cg_cur, ctile, lane);
                     if (cok) ckg = ctile.kg0;
                 }
                 return true;
@@ -602,7 +691,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
                 return true;
             };
-            for (int t = unit; !aborted && next_tile<KIND, false>(p, s_prefix, s_mm, t, gcur, c, lane); t += units) {
+            for (int t = unit; !aborted && next_tile<KIND, CG == 2, CG>(p, s_prefix, s_mm, t, units, gcur, c, lane);
+                 t += units) {
                 if (!wait_warp(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
                 tc_fence_after();  // the epilogue's TMEM reads precede the MMAs below
                 const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
@@ -674,7 +764,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         int gcur = 0;
         int buf = 0;
         Tile c;
-        for (int t = unit; next_tile<KIND, true>(p, s_prefix, s_mm, t, gcur, c, lane); t += units) {
+        for (int t = unit; next_tile<KIND, true, CG>(p, s_prefix, s_mm, t, units, gcur, c, lane); t += units) {
             const int row_coord = c.m_blk * BM * CG + my_rows + 32 * q;
             const int mloc = row_coord + static_cast<int>(lane);
             bool valid;
@@ -689,7 +779,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 const int id = (mloc < p.rows) ? __ldg(p.meta + mloc) : -1;
                 const bool in_range = id >= 0 && id < p.groups;
                 valid = in_range && id == c.g;
-                if (in_range && id != c.g) atomicOr(p.status, DEVERR_MIXED_EXPERT_BLOCK);
+                // a 128-row block must hold one expert (rows of a pair's other
+                // block may belong to another one, written in the other pass)
+                const int own = rank == 0 ? c.e_own[0] : c.e_own[1];
+                if (in_range && id != own) atomicOr(p.status, DEVERR_MIXED_EXPERT_BLOCK);
                 out_row = static_cast<size_t>(mloc);
             }
             // TMA stores clip at the tensor's edges, so for the dense form rows

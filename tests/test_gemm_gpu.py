@@ -220,10 +220,69 @@ def test_contiguous_parity_and_padding(bn):
     assert dg.device_error(clear=True) == 0
 
 
-def test_contiguous_mixed_block_is_flagged():
+CONTIG_PAIR_LAYOUTS = {
+    # experts' 128-row block counts 1, 0, 2, 1, 1 and a padding block: pairs
+    # (0,1) and (2,3) hold two experts each, pair (4,5) one expert and padding
+    "boundaries": dict(counts=[5, 0, 130, 128, 1], tail_blocks=1),
+    # odd block counts everywhere, some experts empty
+    "odd": dict(counts=[300, 0, 129, 640, 1, 0, 257], tail_blocks=0),
+    # an odd number of blocks in total: the last pair's second block is past M
+    "odd_total": dict(counts=[200, 130], tail_blocks=0),
+}
+
+
+@pytest.mark.parametrize("bn", PAIR_BLOCK_NS)
+@pytest.mark.parametrize("layout", sorted(CONTIG_PAIR_LAYOUTS))
+def test_contiguous_parity_cta_pairs(bn, layout):
+    # 256-row pair tiles over 128-row aligned experts: a pair whose blocks
+    # belong to two experts is computed in two passes, one per expert
+    lay = CONTIG_PAIR_LAYOUTS[layout]
+    p = W.contiguous(lay["counts"], 264, 640, seed=17 + bn, tail_blocks=lay["tail_blocks"])
+    dg.set_cta_group(2)
+    d = run_contig(p, bn=bn)
+    check_contig(p, d, what=f"contiguous pairs {layout} bn={bn}")
+    assert dg.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("cg", [1, 2])
+def test_contiguous_beyond_the_block_table(cg):
+    # more 128-row blocks than the kernel keeps experts for in shared memory
+    # (1024): the tile walk reads m_indices directly; sampled outputs and the
+    # sentinel rows are checked
+    counts = [128 * 300 + 5, 128 * 200, 128 * 410 + 77, 128 * 120 + 128]   # 1033 blocks
+    p = W.contiguous(counts, 256, 256, seed=29, tail_blocks=2)
+    assert p["M_total"] // 128 > 1024
+    dg.set_cta_group(cg)
+    d = run_contig(p)
+    assert dg.device_error(clear=True) == 0
+    mi = p["m_indices"]
+    sent = is_sentinel(d)
+    assert sent[mi < 0].all() and not sent[mi >= 0].any()
+    rng = np.random.default_rng(5)
+    rows = rng.choice(np.nonzero(mi >= 0)[0], 256, replace=False)
+    cols = rng.integers(0, p["N"], 256)
+    ref = oracle.m_grouped_fp8_gemm_nt_contiguous_sampled(p["a"], _oracle_pack(p["sfa_f32"]), p["b"],
+                                                          _oracle_pack(p["sfb_f32"]), mi, rows, cols)
+    got = bf16_to_f64(d)[rows, cols]
+    check_fp(got, ref, f"contiguous, {p['M_total'] // 128} blocks, cg={cg}")
+
+
+def test_contiguous_pairs_leading_padding_block():
+    p = W.contiguous([128, 300], 256, 512, seed=23)
+    mi = p["m_indices"].copy()
+    mi[0:128] = -1            # the first pair's first block holds padding only
+    dg.set_cta_group(2)
+    d = run_contig(p, m_indices=mi)
+    check_contig(p, d, m_indices=mi, what="contiguous pairs, leading padding block")
+    assert dg.device_error(clear=True) == 0
+
+
+@pytest.mark.parametrize("cg", [1, 2])
+def test_contiguous_mixed_block_is_flagged(cg):
     p = W.contiguous([100, 100], 128, 256, seed=22)
     mi = p["m_indices"].copy()
     mi[40:60] = 1  # expert 1 inside expert 0's first block
+    dg.set_cta_group(cg)
     d = run_contig(p, m_indices=mi)
     assert dg.device_error(clear=True) & dg.DEVERR_MIXED_EXPERT_BLOCK
     # the block's rows of the larger index are computed, the others untouched
