@@ -75,6 +75,14 @@ const bool g_log = [] {
     const char* v = std::getenv("DGB200_LOG");
     return v != nullptr && v[0] == '1';
 }();
+// Kernels are launched with programmatic stream serialization: a launch may
+// start while the previous kernel in the stream drains; each kernel waits for
+// it (griddepcontrol.wait) before touching global memory. DGB200_PDL=0 turns
+// this off (plain stream order).
+const bool g_pdl = [] {
+    const char* v = std::getenv("DGB200_PDL");
+    return !(v != nullptr && v[0] == '0');
+}();
 // DGB200_K_ROTATE=1 makes every tile start its K walk at a rotated group (default: in order).
 const int g_k_rotate = [] {
     const char* v = std::getenv("DGB200_K_ROTATE");
@@ -389,6 +397,22 @@ double split_bytes(const TileChoice& c, long long m128_blocks, int n) {
     return static_cast<double>(tiles) * c.splits * dg::BM * c.entry->bn * sizeof(float);
 }
 
+// Launch configuration of the elementwise pack kernels (programmatic
+// serialization as for the GEMMs); `attr` must outlive the launch call.
+cudaLaunchConfig_t small_launch(unsigned blocks, int threads, void* stream, cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    if (g_pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cfg;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 dg_status check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* d, int N,
@@ -437,17 +461,26 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     const int units = static_cast<int>(tiles < choice.units ? tiles : choice.units);
     void* args[] = {&p};
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(cg);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    unsigned nattr = 0;
+    if (cg == 2) {
+        attr[nattr].id = cudaLaunchAttributeClusterDimension;
+        attr[nattr].val.clusterDim.x = 2;
+        attr[nattr].val.clusterDim.y = 1;
+        attr[nattr].val.clusterDim.z = 1;
+        ++nattr;
+    }
+    if (g_pdl) {
+        attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[nattr].val.programmaticStreamSerializationAllowed = 1;
+        ++nattr;
+    }
     cfg.gridDim = dim3(static_cast<unsigned>(units * cg));
     cfg.blockDim = dim3(dg::NUM_THREADS);
     cfg.dynamicSmemBytes = static_cast<size_t>(e->smem);
     cfg.stream = static_cast<cudaStream_t>(stream);
     cfg.attrs = attr;
-    cfg.numAttrs = cg == 2 ? 1 : 0;
+    cfg.numAttrs = nattr;
     if (g_log)
         std::fprintf(stderr,
                      "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d splits=%d grid=%d (units %d) smem=%d\n",
@@ -670,15 +703,17 @@ dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int cols, v
     int64_t blocks = (words + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(st->sms) * 8;
     if (blocks > cap) blocks = cap;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = small_launch(static_cast<unsigned>(blocks), threads, stream, attr);
+    cudaError_t err;
     if (cols % 4 == 0 && aligned(sf, 16)) {
-        dg::pack_ue8m0_vec4_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(
-            reinterpret_cast<const float4*>(sf), reinterpret_cast<uint32_t*>(packed), words);
+        err = cudaLaunchKernelEx(&cfg, dg::pack_ue8m0_vec4_kernel, reinterpret_cast<const float4*>(sf),
+                                 reinterpret_cast<uint32_t*>(packed), words);
     } else {
-        dg::pack_ue8m0_rows_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(
-            sf, reinterpret_cast<uint32_t*>(packed), rows, cols, kp);
+        err = cudaLaunchKernelEx(&cfg, dg::pack_ue8m0_rows_kernel, sf, reinterpret_cast<uint32_t*>(packed), rows, cols,
+                                 kp);
     }
-    return cudaPeekAtLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
 dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* bad_count, void* stream) {
@@ -694,8 +729,10 @@ dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* 
     int64_t blocks = (n + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(st->sms) * 8;
     if (blocks > cap) blocks = cap;
-    dg::pack_ue8m0_validate_kernel<<<static_cast<unsigned>(blocks), threads, 0, cs>>>(sf, n, bad_count);
-    return cudaPeekAtLastError() == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = small_launch(static_cast<unsigned>(blocks), threads, stream, attr);
+    const cudaError_t err = cudaLaunchKernelEx(&cfg, dg::pack_ue8m0_validate_kernel, sf, n, bad_count);
+    return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -9,6 +9,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace dg {
 
 __device__ __forceinline__ uint32_t ue8m0_byte(float x) {
@@ -18,6 +20,8 @@ __device__ __forceinline__ uint32_t ue8m0_byte(float x) {
 // cols % 4 == 0 and 16-byte aligned input: word i packs floats 4i..4i+3, so the
 // whole tensor is one flat stream of float4 -> int32.
 __global__ void pack_ue8m0_vec4_kernel(const float4* __restrict__ sf, uint32_t* __restrict__ out, int64_t words) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
         const float4 v = __ldg(sf + i);
@@ -28,6 +32,8 @@ __global__ void pack_ue8m0_vec4_kernel(const float4* __restrict__ sf, uint32_t* 
 // General layout: rows x cols floats -> rows x kp words, zero bytes past cols.
 __global__ void pack_ue8m0_rows_kernel(const float* __restrict__ sf, uint32_t* __restrict__ out, int64_t rows,
                                        int cols, int kp) {
+    griddep_wait();
+    griddep_launch_dependents();
     const int64_t words = rows * kp;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
@@ -46,6 +52,8 @@ __global__ void pack_ue8m0_rows_kernel(const float* __restrict__ sf, uint32_t* _
 
 // Counts scales whose sign bit is set or whose mantissa is non-zero.
 __global__ void pack_ue8m0_validate_kernel(const float* __restrict__ sf, int64_t n, int32_t* __restrict__ bad) {
+    griddep_wait();
+    griddep_launch_dependents();
     int local = 0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {

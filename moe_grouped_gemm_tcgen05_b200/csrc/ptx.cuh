@@ -29,6 +29,19 @@ __device__ __forceinline__ bool elect_one() {
     return pred != 0;
 }
 
+// Programmatic dependent launch. wait: block until the grids this launch
+// depends on have completed and their memory is visible (returns at once when
+// the launch has no such dependency). launch_dependents: allow the next
+// dependent launch in the stream to start (it still waits for this grid's
+// completion before touching memory, if it was built the same way).
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier --
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
