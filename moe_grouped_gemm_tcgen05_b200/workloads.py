@@ -19,6 +19,8 @@ Workloads (seed = 1000 + workload number, numpy PCG64):
   2  contiguous, 8 experts, rows per expert U{3072..5120} padded to 128, N=4096, K=7168
   3  masked, 32 groups, max_m=256, masked_m U{67..124}; up (4096,7168), down (7168,2048)
   4  masked, 256 groups, max_m=512, masked_m ~ Zipf(1.1) on {0..512}, (7168,2048)
+BF16 masked problems (masked_bf16 / masked_bf16_t) use workload 3's shapes and
+masked_m with plain bf16 operands.
 """
 
 from __future__ import annotations
@@ -183,6 +185,34 @@ def workload4():
     return masked(mm, 512, 7168, 2048, seed=1004, fill_invalid_nan=False)
 
 
+# ---- BF16 masked problems ---------------------------------------------------
+#
+# Operands of the BF16 masked grouped GEMM are plain bf16 values (no scales):
+# N(0,1) draws rounded to bf16 (round to nearest even on the fp32 bit
+# pattern), stored as uint16 bit patterns. Rows past masked_m hold a NaN
+# pattern so that a kernel that reads them would be caught.
+
+BF16_NAN = 0x7FC1
+
+
+def _to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def masked_bf16(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bool = True):
+    """BF16 masked M-grouped problem: a [G,max_m,K], b [G,N,K] as uint16 bf16 bits."""
+    rng = rng_for(seed)
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = masked_m.shape[0]
+    a = _to_bf16_bits(_normal(rng, (G, max_m, K)))
+    if fill_invalid_nan:
+        rows = np.arange(max_m)[None, :] >= np.clip(masked_m, 0, max_m)[:, None]
+        a[rows] = BF16_NAN
+    b = _to_bf16_bits(_normal(rng, (G, N, K)))
+    return dict(a=a, b=b, masked_m=masked_m, G=G, max_m=max_m, N=N, K=K)
+
+
 # ---- device-side generation for full-size workloads ------------------------
 #
 # Same recipe as above (N(0,1) draws, power-of-two block scales from the block
@@ -265,6 +295,17 @@ def masked_t(masked_m, max_m: int, N: int, K: int, seed: int, device="cuda"):
     b, sfb = grouped_weights_t(g, G, N, K, device)
     return dict(a=a.view(G, max_m, K), sfa_f32=sfa.view(G, max_m, K // BLOCK), b=b, sfb_f32=sfb,
                 masked_m=torch.from_numpy(masked_m).to(device), masked_m_host=masked_m,
+                G=G, max_m=max_m, N=N, K=K)
+
+
+def masked_bf16_t(masked_m, max_m: int, N: int, K: int, seed: int, device="cuda"):
+    """BF16 masked problem drawn on the device (torch bfloat16 tensors)."""
+    masked_m = np.asarray(masked_m, dtype=np.int32)
+    G = masked_m.shape[0]
+    g = _gen(device, seed)
+    a = torch.randn((G, max_m, K), generator=g, device=device).to(torch.bfloat16)
+    b = torch.randn((G, N, K), generator=g, device=device).to(torch.bfloat16)
+    return dict(a=a, b=b, masked_m=torch.from_numpy(masked_m).to(device), masked_m_host=masked_m,
                 G=G, max_m=max_m, N=N, K=K)
 
 

@@ -11,11 +11,12 @@ Everything is numpy in float64.
 Modules
 -------
 fp8    -- the OCP E4M3 value table (``e4m3_to_f64``)
+bf16   -- bf16 operand values (``bf16_to_f64``)
 ue8m0  -- UE8M0 scale bytes: decode, the capture-safe pack of fp32 scales
           into four bytes per int32, the matching unpack, and the optional
           eager validator
 gemm   -- dequantise-and-multiply references for the dense NT GEMM and the
-          contiguous / masked M-grouped GEMMs
+          contiguous / masked M-grouped GEMMs, and the BF16 masked grouped GEMM
 
 Sources (web pages about DeepGEMM):
   [P1] "DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs:
@@ -28,6 +29,7 @@ Every function names the section it follows.
 """
 
 from .fp8 import e4m3_to_f64, E4M3_MAX  # noqa: F401
+from .bf16 import bf16_to_f64  # noqa: F401
 from .ue8m0 import (  # noqa: F401
     ue8m0_to_f64,
     pack_ue8m0,
@@ -45,4 +47,6 @@ from .gemm import (  # noqa: F401
     m_grouped_fp8_gemm_nt_masked,
     m_grouped_fp8_gemm_nt_masked_sampled,
     masked_valid_rows,
+    m_grouped_bf16_gemm_nt_masked,
+    m_grouped_bf16_gemm_nt_masked_sampled,
 )

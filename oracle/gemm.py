@@ -34,6 +34,7 @@ whose output is defined; rows outside it must keep their previous bits.
 
 import numpy as np
 
+from .bf16 import bf16_to_f64
 from .fp8 import e4m3_to_f64
 from .ue8m0 import ue8m0_to_f64, unpack_ue8m0
 
@@ -178,3 +179,42 @@ def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb) -> np.ndarray:
     scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))[n_idx // BLOCK]
     B = (e4m3_to_f64(b_rows).reshape(P, KB, BLOCK) * scale[:, :, None]).reshape(P, K)
     return np.einsum("ik,ik->i", A, B)
+
+
+# ---- BF16 masked grouped GEMM ------------------------------------------------
+
+def m_grouped_bf16_gemm_nt_masked(a, b, masked_m):
+    """BF16 masked M-grouped GEMM ("DeepGEMM CUDA Graph Compatibility for Masked
+    Grouped GEMMs", Core Components and Tensor-Based Metadata Arguments).
+
+    a: uint16 bf16 bits [G, max_m, K]; b: uint16 bf16 bits [G, N, K];
+    masked_m: int [G]. For every group g, D[g, :m_g] = A[g, :m_g] . B[g]^T with
+    m_g = clamp(masked_m[g], 0, max_m), in float64 (no scales: the operands are
+    plain bf16 values). Returns (D with NaN on rows outside the valid region,
+    valid [G, max_m])."""
+    a = np.asarray(a, dtype=np.uint16)
+    b = np.asarray(b, dtype=np.uint16)
+    G, max_m, K = a.shape
+    N = b.shape[1]
+    mm = np.clip(np.asarray(masked_m, dtype=np.int64), 0, max_m)
+    out = np.full((G, max_m, N), np.nan)
+    for g in range(G):
+        m = int(mm[g])
+        if m:
+            out[g, :m] = bf16_to_f64(a[g, :m]) @ bf16_to_f64(b[g]).T
+    valid = np.arange(max_m)[None, :] < mm[:, None]
+    return out, valid
+
+
+def m_grouped_bf16_gemm_nt_masked_sampled(a, b, masked_m, groups, rows, cols):
+    """Sampled outputs D[groups[i], rows[i], cols[i]] of the BF16 masked GEMM,
+    one at a time; every sampled row must be inside its group's valid rows."""
+    a = np.asarray(a, dtype=np.uint16)
+    b = np.asarray(b, dtype=np.uint16)
+    mm = np.clip(np.asarray(masked_m, dtype=np.int64), 0, a.shape[1])
+    groups = np.asarray(groups, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    cols = np.asarray(cols, dtype=np.int64)
+    if np.any(rows >= mm[groups]):
+        raise ValueError("sampled rows must be valid rows of their group")
+    return np.einsum("ik,ik->i", bf16_to_f64(a[groups, rows]), bf16_to_f64(b[groups, cols]))

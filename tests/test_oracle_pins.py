@@ -335,3 +335,127 @@ def test_points_match_full():
     c = rng.integers(0, N, size=40)
     pts = oracle.fp8_gemm_nt_points(a[r], sfa[r], b[c], c, sfb)
     np.testing.assert_allclose(pts, full[r, c], rtol=1e-13, atol=0)
+
+
+# ------------------------------------------------------ BF16 masked GEMM ----
+
+def torch_bf16(bits):
+    """torch's bfloat16 decode of uint16 bit patterns, as float64 (library routine)."""
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(bits, dtype=np.uint16)).view(np.int16))
+    return t.view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def test_bf16_spot_values_from_binary32_layout():
+    # sign | 8-bit exponent (bias 127) | 7-bit fraction
+    cases = {0x3F80: 1.0, 0xC000: -2.0, 0x3FC0: 1.5, 0x4049: 3.140625, 0x0000: 0.0,
+             0x0001: 2.0 ** -133, 0x0080: 2.0 ** -126, 0x7F7F: (2 - 2.0 ** -7) * 2.0 ** 127}
+    got = oracle.bf16_to_f64(np.array(list(cases), dtype=np.uint16))
+    assert got.tolist() == list(cases.values())
+    assert np.isinf(oracle.bf16_to_f64(np.array([0x7F80], np.uint16)))[0]
+    assert np.isnan(oracle.bf16_to_f64(np.array([0x7FC0], np.uint16)))[0]
+
+
+def test_bf16_decode_matches_torch_for_every_code():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    mine, ref = oracle.bf16_to_f64(codes), torch_bf16(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(mine), nan)
+    assert np.array_equal(mine[~nan], ref[~nan])
+
+
+def _bf16_bits_of(vals):
+    """Exact bf16 bit patterns of values that bf16 represents (a test helper)."""
+    u = np.asarray(vals, dtype=np.float32).view(np.uint32)
+    assert (u & 0xFFFF == 0).all()
+    return (u >> 16).astype(np.uint16)
+
+
+def test_bf16_masked_equals_exact_rational_brute_force():
+    rng = np.random.default_rng(12)
+    G, max_m, N, K = 3, 5, 4, 16
+    # values m * 2^e with 8-bit m and a narrow exponent range: every product
+    # and partial sum is exact in float64, so the oracle must equal the
+    # rational sum exactly
+    def draw(shape):
+        m = rng.integers(-255, 256, size=shape)
+        e = rng.integers(-8, 0, size=shape)
+        return _bf16_bits_of((m * np.ldexp(1.0, e)).astype(np.float32))
+    a, b = draw((G, max_m, K)), draw((G, N, K))
+    masked_m = np.array([5, 2, 0], dtype=np.int32)
+    d, valid = oracle.m_grouped_bf16_gemm_nt_masked(a, b, masked_m)
+    av, bv = torch_bf16(a), torch_bf16(b)
+    for g in range(G):
+        for m in range(max_m):
+            for n in range(N):
+                if m < masked_m[g]:
+                    exact = sum(Fraction(float(av[g, m, k])) * Fraction(float(bv[g, n, k])) for k in range(K))
+                    assert Fraction(d[g, m, n]) == exact
+                else:
+                    assert not valid[g, m] and np.isnan(d[g, m, n])
+
+
+def bf16_one_hot_check(fn) -> bool:
+    """One-hot A rows pick one column of B exactly: D[g, m, n] = B[g, n, k_m]."""
+    rng = np.random.default_rng(13)
+    G, max_m, N, K = 2, 6, 40, 192
+    ks = np.array([0, 63, 64, 100, 150, 191])
+    a = np.zeros((G, max_m, K), dtype=np.uint16)
+    a[:, np.arange(max_m), ks] = 0x3F80
+    b = rng.integers(0, 0x7F00, size=(G, N, K)).astype(np.uint16) | (rng.integers(0, 2, size=(G, N, K)) << 15).astype(np.uint16)
+    masked_m = np.array([6, 4], dtype=np.int32)
+    d, valid = fn(a, b, masked_m)
+    bv = torch_bf16(b)
+    for g in range(G):
+        for m in range(int(masked_m[g])):
+            if not np.array_equal(d[g, m], bv[g, :, ks[m]]):
+                return False
+    return bool(valid[1, :4].all() and not valid[1, 4:].any())
+
+
+def test_bf16_masked_one_hot_exact():
+    assert bf16_one_hot_check(oracle.m_grouped_bf16_gemm_nt_masked)
+
+
+def test_bf16_masked_clamp_and_sampled():
+    rng = np.random.default_rng(14)
+    G, max_m, N, K = 4, 7, 30, 64
+    a = rng.integers(0x3C00, 0x4000, size=(G, max_m, K)).astype(np.uint16)
+    b = rng.integers(0x3C00, 0x4000, size=(G, N, K)).astype(np.uint16)
+    masked_m = np.array([3, -2, 50, 0], dtype=np.int32)
+    d, valid = oracle.m_grouped_bf16_gemm_nt_masked(a, b, masked_m)
+    assert valid.sum(axis=1).tolist() == [3, 0, max_m, 0]
+    # the whole valid region is a plain library matmul of the decoded values
+    for g in range(G):
+        m = int(valid[g].sum())
+        if m:
+            ref = (torch.from_numpy(torch_bf16(a[g, :m])) @ torch.from_numpy(torch_bf16(b[g])).T).numpy()
+            np.testing.assert_allclose(d[g, :m], ref, rtol=1e-13, atol=0)
+    gs = np.array([0, 0, 2, 2]); rs = np.array([0, 2, 6, 1]); cs = np.array([5, 29, 0, 17])
+    assert np.array_equal(oracle.m_grouped_bf16_gemm_nt_masked_sampled(a, b, masked_m, gs, rs, cs), d[gs, rs, cs])
+
+
+def _planted_bf16(kind):
+    """A copy of the BF16 masked oracle with one plausible mistake planted (CPU only)."""
+    def fn(a, b, masked_m):
+        G, max_m, K = a.shape
+        mm = np.clip(masked_m, 0, max_m)
+        if kind == "rows_off_by_one":
+            mm = np.clip(masked_m + 1, 0, max_m)
+        out = np.full((G, max_m, b.shape[1]), np.nan)
+        for g in range(G):
+            m = int(mm[g])
+            A = oracle.bf16_to_f64(a[g, :m])
+            B = oracle.bf16_to_f64(b[g])
+            if kind == "half_swapped":   # low and high bytes of each code swapped
+                B = oracle.bf16_to_f64(((b[g] >> 8) | (b[g] << 8)).astype(np.uint16))
+            if kind == "wrong_group":
+                B = oracle.bf16_to_f64(b[(g + 1) % G])
+            out[g, :m] = A @ B.T
+        valid = np.arange(max_m)[None, :] < mm[:, None]
+        return out, valid
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["rows_off_by_one", "half_swapped", "wrong_group"])
+def test_bf16_pins_catch_planted_mistakes(kind):
+    assert not bf16_one_hot_check(_planted_bf16(kind)), kind
