@@ -386,6 +386,43 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
     masked_case("masked_zipf_256g_7168x2048_pack+gemm", p, True,
                 lambda r: W.zipf_masked_m(W.rng_for(6000 + r)))
     del p
+
+    # BF16 masked decode (same shapes and masked_m draws, plain bf16 operands)
+    def masked_bf16_case(name, q, rng):
+        G, max_m, N, K = q["G"], q["max_m"], q["N"], q["K"]
+        d = torch.empty((G, max_m, N), dtype=torch.bfloat16, device=dev)
+        draws = [q["masked_m_host"]] + [rng(r) for r in range(1, reps)]
+        pool = torch.from_numpy(np.stack(draws).astype(np.int32)).to(dev)
+        mm = q["masked_m"]
+        ops = []
+        for r in range(reps):
+            def op(r=r):
+                mm.copy_(pool[r])
+                dg.m_grouped_bf16_gemm_nt_masked(q["a"], q["b"], d, mm)
+            ops.append(op)
+        ops[0]()
+        torch.cuda.synchronize()
+        g = EventGraph(ops)
+        g.replay()
+        torch.cuda.synchronize()
+        durs = g.durations_ms()
+        g.close()
+        gbs, fr = [], []
+        for r, ms in enumerate(durs):
+            m = np.clip(draws[r], 0, max_m)
+            rows, gnz = int(m.sum()), int((m > 0).sum())
+            by = 2 * rows * K + 2 * gnz * N * K + 2 * rows * N + 4 * G
+            gbs.append(by / ms / 1e6)
+            fr.append(by / (peaks["hbm"] * 1e9) / (ms * 1e-3))
+        out[name] = {"us": statistics.median(durs) * 1e3, "GB/s": statistics.median(gbs),
+                     "roofline_frac": statistics.median(fr), "bound": "hbm", "calls": reps}
+
+    for proj in ("up", "down"):
+        N, K = (4096, 7168) if proj == "up" else (7168, 2048)
+        q = W.masked_bf16_t(W.masked_m_uniform(W.rng_for(1003)), 256, N, K, seed=1003, device=dev)
+        masked_bf16_case(f"masked_bf16_decode_32g_{proj}_{N}x{K}", q,
+                         lambda r: W.masked_m_uniform(W.rng_for(5000 + r)))
+        del q
     torch.cuda.empty_cache()
     return out
 

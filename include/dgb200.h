@@ -232,6 +232,24 @@ DG_API dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa,
                                        int G, int max_m, int N, int K, void* stream);
 
 /*
+ * Masked M-grouped BF16 GEMM ("DeepGEMM CUDA Graph Compatibility for Masked
+ * Grouped GEMMs", Core Components: the BF16 masked grouped GEMM kernel, and
+ * Tensor-Based Metadata Arguments). Plain bf16 operands, no scales; fp32
+ * accumulation, bf16 output.
+ *   a        : device, bf16 [G, max_m, K]
+ *   b        : device, bf16 [G, N, K]
+ *   d        : device, bf16 [G, max_m, N]
+ *   masked_m : device, int32 [G]; group g uses its first masked_m[g] rows,
+ *              clamped on the device to [0, max_m].
+ * Limits: K % 64 == 0 (one 128-byte row of K per pipeline stage), N % 8 == 0,
+ * G <= 1024, a / b / d 16-byte aligned. Rows at or beyond masked_m[g] are never
+ * written (a pre-filled sentinel survives). The grid depends only on
+ * (G, max_m, N, K); the call is capture safe like the FP8 masked GEMM.
+ */
+DG_API dg_status m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d, const int32_t* masked_m, int G,
+                                               int max_m, int N, int K, void* stream);
+
+/*
  * Capture-safe UE8M0 pack ("[GH-ISSUE #414] pack_ue8m0_to_int is not CUDA Graph
  * capture safe", Expected behavior). For fp32 scales sf [rows, cols] writes
  * packed [rows, ceil(cols/4)] int32 with byte (bits(sf[r][c]) >> 23) & 0xFF at

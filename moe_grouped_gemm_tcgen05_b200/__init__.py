@@ -24,7 +24,7 @@ __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
-    "fp8_gemm_nt_noalloc",
+    "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -85,6 +85,8 @@ def load():
         L.dgb200_set_test_hooks.argtypes = [i32, i32]
         L.fp8_gemm_nt.restype = i32
         L.fp8_gemm_nt.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
+        L.m_grouped_bf16_gemm_nt_masked.restype = i32
+        L.m_grouped_bf16_gemm_nt_masked.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.fp8_gemm_nt_noalloc.restype = i32
         L.fp8_gemm_nt_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_contiguous.restype = i32
@@ -239,6 +241,24 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, max_m=None):
     _check("m_grouped_fp8_gemm_nt_masked",
            load().m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m),
                                                G, max_m, N, K, _stream()))
+    return d
+
+
+_BF16_OPERAND = (torch.bfloat16, torch.int16, torch.uint16)  # bf16 values or their bit patterns
+
+
+def m_grouped_bf16_gemm_nt_masked(a, b, d, masked_m):
+    """Masked M-grouped BF16 GEMM: d[g, :m_g] = a[g, :m_g] @ b[g]^T, m_g = masked_m[g] (device)."""
+    _need(a, "a", _BF16_OPERAND)
+    G, max_m, K = a.shape
+    _need(b, "b", _BF16_OPERAND)
+    N = b.shape[1]
+    _need(b, "b", _BF16_OPERAND, (G, N, K))
+    _need(d, "d", _BF16, (G, max_m, N))
+    _need(masked_m, "masked_m", _I32, (G,))
+    _check("m_grouped_bf16_gemm_nt_masked",
+           load().m_grouped_bf16_gemm_nt_masked(_ptr(a), _ptr(b), _ptr(d), _ptr(masked_m), G, max_m, N, K,
+                                                _stream()))
     return d
 
 

@@ -91,23 +91,26 @@ const int g_k_rotate = [] {
 
 // --------------------------------------------------------------- kernels ----
 
-template <int BN, int KIND, int CG>
+template <int BN, int KIND, int CG, int DT>
 void* kernel_ptr() {
-    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG>);
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT>);
 }
 
 struct KernelEntry {
     int bn;
     int kind;
-    int cg;     // CTAs per MMA unit (1, or a cluster pair)
+    int cg;      // CTAs per MMA unit (1, or a cluster pair)
+    int dt;      // operand type (dg::kE4M3 block-scaled, dg::kBF16)
     void* fn;
     int smem;
     int stages;  // depth of the operand ring
 };
 
-#define DG_ENTRY(BN, KIND, CG)                                                                 \
-    {BN, KIND, CG, kernel_ptr<BN, KIND, CG>(), dg::GemmConfig<BN, CG, dg::sched_ints<KIND>()>::SMEM_BYTES, \
-     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>()>::STAGES}
+#define DG_ENTRY_T(BN, KIND, CG, DT)                                                                            \
+    {BN, KIND, CG, DT, kernel_ptr<BN, KIND, CG, DT>(),                                                          \
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES}
+#define DG_ENTRY(BN, KIND, CG) DG_ENTRY_T(BN, KIND, CG, dg::kE4M3)
+#define DG_BF16_MASKED(BN) DG_ENTRY_T(BN, dg::kMasked, 1, dg::kBF16)
 #define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1)
 
 const KernelEntry kKernels[] = {
@@ -117,6 +120,8 @@ const KernelEntry kKernels[] = {
     DG_ENTRY(224, dg::kDense, 2), DG_ENTRY(256, dg::kDense, 2),
     DG_ENTRY(128, dg::kContiguous, 2), DG_ENTRY(160, dg::kContiguous, 2), DG_ENTRY(192, dg::kContiguous, 2),
     DG_ENTRY(224, dg::kContiguous, 2), DG_ENTRY(256, dg::kContiguous, 2),
+    DG_BF16_MASKED(64), DG_BF16_MASKED(96), DG_BF16_MASKED(128), DG_BF16_MASKED(160),
+    DG_BF16_MASKED(192), DG_BF16_MASKED(224), DG_BF16_MASKED(256),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
@@ -230,14 +235,18 @@ dg_status current_device(DeviceState** out) {
 
 // ------------------------------------------------------------ tensor maps --
 
-bool encode_kmajor_u8(CUtensorMap* map, const void* base, int rank, uint64_t k, uint64_t rows, uint64_t mats,
-                      uint32_t box_rows) {
+// K-major operand (k values per row) of 1-byte (E4M3) or 2-byte (BF16)
+// elements; the box is one 128-byte row of K by `box_rows` rows.
+bool encode_kmajor(CUtensorMap* map, const void* base, int rank, uint64_t k, uint64_t rows, uint64_t mats,
+                   uint32_t box_rows, int dt) {
+    const uint64_t esz = dt == dg::kBF16 ? 2 : 1;
     cuuint64_t dims[3] = {k, rows, mats};
-    cuuint64_t strides[2] = {k, k * rows};  // bytes, dims 1..rank-1
-    cuuint32_t box[3] = {128, box_rows, 1};
+    cuuint64_t strides[2] = {k * esz, k * esz * rows};  // bytes, dims 1..rank-1
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / esz), box_rows, 1};
     cuuint32_t elem[3] = {1, 1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
-                          dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUtensorMapDataType type = dt == dg::kBF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    CUresult r = g_encode(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -315,8 +324,8 @@ struct SplitScratch {
 };
 
 TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                          long long unique_bytes, int forced_splits, const SplitScratch& scratch) {
-    const int kb = k / 128;
+                          long long unique_bytes, int forced_splits, const SplitScratch& scratch, int dt = dg::kE4M3) {
+    const int kb = k / (dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K (one pipeline stage each)
     const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
     const int forced_cg = kind != dg::kMasked ? g_force_cg.load() : 0;  // no pairs for the masked form
@@ -325,7 +334,7 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
-        if (e.kind != kind) continue;
+        if (e.kind != kind || e.dt != dt) continue;
         if (forced_bn != 0 && e.bn != forced_bn) continue;
         if (forced_cg != 0 && e.cg != forced_cg) continue;
         if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
@@ -384,10 +393,10 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
 // The library's own choice: the allocated split-K workspace, and the split
 // count forced by dgb200_set_splits (dense form).
 TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                       long long unique_bytes) {
+                       long long unique_bytes, int dt = dg::kE4M3) {
     const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
     const SplitScratch scratch{st->split_ws != nullptr, static_cast<double>(kSplitWsBytes), kSplitCounters};
-    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch);
+    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt);
 }
 
 // Bytes of split-K partials a choice writes (0 when it does not split).
@@ -437,7 +446,7 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     const int bn = e->bn;
     const int cg = e->cg;
     p.status = st->status;
-    p.kb = p.k / 128;
+    p.kb = p.k / (e->dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K per operand row
     p.kp = (p.kb + 3) / 4;
     p.nb_sf = (p.n + 127) / 128;
     p.num_n_blocks = (p.n + bn - 1) / bn;
@@ -449,9 +458,10 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.ws = choice.splits > 1 ? ws : nullptr;
     p.counters = choice.splits > 1 ? counters : nullptr;
     p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
-    if (!encode_kmajor_u8(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128)) return DG_ERR_INVALID_ARG;
-    if (!encode_kmajor_u8(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats,
-                          static_cast<uint32_t>(bn / cg)))
+    if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128, e->dt))
+        return DG_ERR_INVALID_ARG;
+    if (!encode_kmajor(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn / cg),
+                       e->dt))
         return DG_ERR_INVALID_ARG;
     if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
     // contiguous pairs walk two passes (see next_tile in gemm_kernel.cuh)
@@ -491,8 +501,9 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
 
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
                       long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
-                      int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats) {
-    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes);
+                      int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats,
+                      int dt = dg::kE4M3) {
+    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt);
     return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
                             a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
 }
@@ -689,6 +700,31 @@ dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const 
     const long long bytes = static_cast<long long>(G) * N * K;  // the weights; the valid rows are unknown here
     return launch_gemm(dg::kMasked, p, mb_total, mb_total, bytes, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
                        static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+}
+
+dg_status m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d, const int32_t* masked_m, int G,
+                                        int max_m, int N, int K, void* stream) {
+    if (!a || !b || !d || !masked_m) return DG_ERR_INVALID_ARG;
+    if (G <= 0 || max_m <= 0 || N <= 0 || K <= 0) return DG_ERR_INVALID_ARG;
+    if (K % 64 != 0 || N % 8 != 0) return DG_ERR_INVALID_ARG;
+    if (G > dg::MAX_MASKED_GROUPS) return DG_ERR_UNSUPPORTED;
+    if (!aligned(a, 16) || !aligned(b, 16) || !aligned(d, 16) || !aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    dg_status s = current_device(&st);
+    if (s != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = masked_m;
+    p.rows = max_m;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (max_m + dg::BM - 1) / dg::BM;
+    const long long mb_total = static_cast<long long>(G) * p.num_m_blocks;
+    const long long bytes = 2LL * G * N * K;  // the weights; the valid rows are unknown here
+    return launch_gemm(dg::kMasked, p, mb_total, mb_total, bytes, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
+                       static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G), dg::kBF16);
 }
 
 dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int cols, void* stream) {

@@ -69,10 +69,11 @@
 namespace dg {
 
 enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+// Operand type: E4M3 with packed UE8M0 block scales, or plain BF16 (no scales).
+enum OperandType : int { kE4M3 = 0, kBF16 = 1 };
 
 constexpr int BM = 128;                 // rows of A per CTA
-constexpr int BK = 128;                 // K per pipeline stage = one scale block
-constexpr int MMA_K = 32;               // K of one kind::mxf8f6f4 MMA
+constexpr int BK = 128;                 // bytes of K per pipeline stage (E4M3: 128 values = one scale block)
 constexpr int NUM_THREADS = 224;
 constexpr int SF_RING = 4;              // scale-word groups in flight
 constexpr int MAX_MASKED_GROUPS = 1024;
@@ -119,7 +120,7 @@ __host__ __device__ constexpr int sched_ints() {
     return KIND == kMasked ? 2 * MAX_MASKED_GROUPS + 8 : (KIND == kContiguous ? MAX_CACHED_BLOCKS + 8 : 16);
 }
 
-template <int BN, int CG, int SCHED_INTS>
+template <int BN, int CG, int SCHED_INTS, int DT = kE4M3>
 struct GemmConfig {
     static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 32 in [32, 256]");
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
@@ -129,7 +130,7 @@ struct GemmConfig {
     static constexpr int SFB_CHUNKS = (BN + 127) / 128;         // 128-column chunks of B scales (full width)
     static constexpr int SFA_BYTES = 512;                       // 32 rows x 16 bytes
     static constexpr int SFB_BYTES = 512 * SFB_CHUNKS;
-    static constexpr int SF_SLOT_BYTES = SFA_BYTES + SFB_BYTES;  // one group of scale words
+    static constexpr int SF_SLOT_BYTES = DT == kE4M3 ? SFA_BYTES + SFB_BYTES : 0;  // one group of scale words
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr uint32_t TX_BYTES = CG * (A_BYTES + B_BYTES);  // TMA bytes per stage, both CTAs
     static constexpr int EPI_WARP_BYTES = 2 * 2048;             // two 32x32 bf16 staging buffers per warp
@@ -147,12 +148,14 @@ struct GemmConfig {
     // alternate groups so that the copy of the next group's scales never
     // overwrites words that MMAs still in the pipe are reading.
     static constexpr int ACC_COLS = BN;
-    static constexpr int SF_COLS = 4 + 4 * SFB_CHUNKS;
+    static constexpr int SF_COLS = DT == kE4M3 ? 4 + 4 * SFB_CHUNKS : 0;
     static constexpr int NUM_ACC = (2 * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1;
     static constexpr int SF_BASE = NUM_ACC * ACC_COLS;
     static_assert(SF_BASE + 2 * SF_COLS <= 512, "TMEM overflow");
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t IDESC = idesc_mxf8_e4m3_ue8m0(BM * CG, BN);
+    static constexpr uint32_t IDESC = DT == kE4M3 ? idesc_mxf8_e4m3_ue8m0(BM * CG, BN) : idesc_bf16_f32(BM * CG, BN);
+    // K values per 128-byte row of a stage and per MMA instruction
+    static constexpr int K_PER_STAGE = DT == kE4M3 ? 128 : 64;
 };
 
 struct Tile {
@@ -385,10 +388,11 @@ struct ScaleWords {
 
 // ------------------------------------------------------------------ kernel --
 
-template <int BN, int KIND, int CG>
+template <int BN, int KIND, int CG, int DT>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
     static_assert(CG == 1 || KIND != kMasked, "CTA pairs are built for the dense and contiguous forms");
-    using Cfg = GemmConfig<BN, CG, sched_ints<KIND>()>;
+    static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
+    using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT>;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int NUM_ACC = Cfg::NUM_ACC;
 
@@ -549,7 +553,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 if (elect_one()) {
                     uint8_t* a_dst = smem_a + stage * Cfg::A_BYTES;
                     uint8_t* b_dst = smem_b + stage * Cfg::B_BYTES;
-                    const int kx = kb * BK;
+                    const int kx = kb * Cfg::K_PER_STAGE;  // TMA coordinates are in elements
                     if constexpr (CG == 1) {
                         mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
                         if constexpr (KIND == kMasked) {
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         // For a pair the leader's warp gathers the words of both CTAs and writes
         // the peer's share into the peer's shared memory, so the hand-off to the
         // MMA warp stays inside the leader CTA; the peer's warp has no work.
-        if (CG == 1 || leader) {
+        if (DT == kE4M3 && (CG == 1 || leader)) {
             [[maybe_unused]] uint32_t peer_sf0 = 0;  // the peer's scale ring (pairs)
             if constexpr (CG == 2) peer_sf0 = mapa_shared(smem_u32(smem_sf), 1);
             // Groups are visited in the MMA warp's order (tile by tile, K groups
@@ -682,6 +686,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // next group's scale words (both CTAs of a pair) -> TMEM at `dst`;
             // the ring slot is free again once the copy has completed
             auto copy_scales = [&](uint32_t dst) -> bool {
+                if constexpr (DT != kE4M3) return true;  // plain BF16 operands carry no scales
                 if (!wait_warp(&sf_full_bar[slot], sf_phase, p, s_abort)) return false;
                 tc_fence_after();
                 if (elect_one()) {
@@ -724,12 +729,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         const uint64_t adesc = smem_desc_sw128(smem_u32(smem_a + stage * Cfg::A_BYTES));
                         const uint64_t bdesc = smem_desc_sw128(smem_u32(smem_b + stage * Cfg::B_BYTES));
                         if (elect_one()) {
+                            // four MMAs per 128-byte row of K: E4M3 K = 32, BF16 K = 16 per instruction;
+                            // each advances the start address by 32 bytes inside the swizzled row
 #pragma unroll
-                            for (int k = 0; k < BK / MMA_K; ++k) {
-                                // advance the start address by 32 bytes of K inside the swizzled row
-                                const uint64_t koff = static_cast<uint64_t>((k * MMA_K) >> 4);
-                                tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
-                                                                sfb_t, (gi > c.kg0 || kb > kb0 || k > 0) ? 1u : 0u);
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t koff = static_cast<uint64_t>((k * 32) >> 4);
+                                const uint32_t accumulate = (gi > c.kg0 || kb > kb0 || k > 0) ? 1u : 0u;
+                                if constexpr (DT == kE4M3)
+                                    tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
+                                                                    sfb_t, accumulate);
+                                else
+                                    tc_mma_f16<CG>(d_tmem, adesc + koff, bdesc + koff, Cfg::IDESC, accumulate);
                             }
                             tc_commit<CG>(&empty_bar[stage]);
                         }

@@ -230,6 +230,27 @@ __device__ __forceinline__ void tc_mma_mxf8f6f4_block_scale(uint32_t d_tmem, uin
             : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T for 16-bit operands (kind::f16, K = 16 per
+// instruction; bf16 or fp16 as the instruction descriptor says).
+template <int CG>
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    if constexpr (CG == 1)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+            ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+            : "memory");
+}
+
 // Arrive once on `bar` (for CG = 2: on the barrier at this offset in both CTAs
 // of the pair) when all previously issued tcgen05 async ops of this thread
 // have completed.
@@ -343,6 +364,15 @@ __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3_ue8m0(uint32_t m, uint32_t n) {
     return ((n >> 3) << 17)      // N >> 3
          | (1u << 23)            // scale format UE8M0
+         | ((m >> 4) << 24);     // M >> 4
+}
+
+// Instruction descriptor of kind::f16: BF16 x BF16 -> F32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t m, uint32_t n) {
+    return (1u << 4)             // D format F32
+         | (1u << 7)             // A format BF16
+         | (1u << 10)            // B format BF16
+         | ((n >> 3) << 17)      // N >> 3
          | ((m >> 4) << 24);     // M >> 4
 }
 
