@@ -181,6 +181,26 @@ def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb) -> np.ndarray:
     return np.einsum("ik,ik->i", A, B)
 
 
+# ---- dense GEMM with an accumulation matrix ------------------------------------
+
+def fp8_gemm_nt_acc(a, sfa, b, sfb, c=None) -> np.ndarray:
+    """D = C + A^ . B^^T in float64 ("DeepInside DeepGEMM", §4 Hands-on Geek
+    Guide: the standard non-grouped FP8 NT GEMM computes D = C + A @ B.T; the
+    example passes C as a bf16 [M, N] tensor and the output dtype).
+
+    c: None (C = 0) or the values of C as a float array [M, N] (decoded from
+    D's storage type by the caller). Readings: C has D's storage type (bf16 or
+    fp32) and is added to the fp32 accumulation before the final conversion,
+    so the reference is the exact sum C + A^.B^^T."""
+    d = fp8_gemm_nt(a, sfa, b, sfb)
+    if c is None:
+        return d
+    c = np.asarray(c, dtype=np.float64)
+    if c.shape != d.shape:
+        raise ValueError(f"C has shape {c.shape}, D has {d.shape}")
+    return c + d
+
+
 # ---- BF16 masked grouped GEMM ------------------------------------------------
 
 def m_grouped_bf16_gemm_nt_masked(a, b, masked_m):

@@ -459,3 +459,45 @@ def _planted_bf16(kind):
 @pytest.mark.parametrize("kind", ["rows_off_by_one", "half_swapped", "wrong_group"])
 def test_bf16_pins_catch_planted_mistakes(kind):
     assert not bf16_one_hot_check(_planted_bf16(kind)), kind
+
+
+# ------------------------------------------- dense GEMM with a C matrix ----
+
+def test_acc_with_zero_or_absent_c_is_the_plain_gemm():
+    rng = np.random.default_rng(21)
+    M, N, K = 17, 140, 384
+    a, b = _rand_codes(rng, (M, K)), _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(rng.integers(120, 135, size=(M, 3)).astype(np.uint8))
+    sfb = _pack_bytes(rng.integers(120, 135, size=(2, 3)).astype(np.uint8))
+    plain = oracle.fp8_gemm_nt(a, sfa, b, sfb)
+    assert np.array_equal(oracle.fp8_gemm_nt_acc(a, sfa, b, sfb), plain)
+    assert np.array_equal(oracle.fp8_gemm_nt_acc(a, sfa, b, sfb, np.zeros((M, N))), plain)
+
+
+def test_acc_with_zero_a_returns_c_exactly():
+    rng = np.random.default_rng(22)
+    M, N, K = 9, 64, 256
+    a = np.zeros((M, K), dtype=np.uint8)
+    b = _rand_codes(rng, (N, K))
+    c = rng.standard_normal((M, N)).astype(np.float32).astype(np.float64)
+    sfa = _pack_bytes(np.full((M, 2), 127, np.uint8))
+    sfb = _pack_bytes(np.full((1, 2), 127, np.uint8))
+    assert np.array_equal(oracle.fp8_gemm_nt_acc(a, sfa, b, sfb, c), c)
+
+
+def test_acc_one_hot_plus_c_exact():
+    # one-hot A rows select one (scaled) column of B; adding a C of small
+    # integers keeps every sum exact in float64
+    rng = np.random.default_rng(23)
+    M, N, K = 4, 130, 256
+    ks = np.array([0, 100, 128, 255])
+    a = np.zeros((M, K), dtype=np.uint8)
+    a[np.arange(M), ks] = 0x38
+    b = _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(np.full((M, 2), 127, np.uint8))
+    sfb = _pack_bytes(np.full((2, 2), 127, np.uint8))
+    c = rng.integers(-8, 9, size=(M, N)).astype(np.float64)
+    got = oracle.fp8_gemm_nt_acc(a, sfa, b, sfb, c)
+    bv = torch_e4m3(b)
+    for m in range(M):
+        assert np.array_equal(got[m], c[m] + bv[:, ks[m]])
