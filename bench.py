@@ -387,6 +387,24 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                 lambda r: W.zipf_masked_m(W.rng_for(6000 + r)))
     del p
 
+    # dense with an accumulation matrix: D (fp32) = C (fp32) + A.B^T, in place
+    M, N, K = 4096, 7168, 16384
+    p = W.workload1_t(M, N, K, dev)
+    sfa, sfb = dg.pack_ue8m0(p["sfa_f32"]), dg.pack_ue8m0(p["sfb_f32"])
+    d = torch.randn((M, N), dtype=torch.float32, device=dev)
+    op = lambda: dg.fp8_gemm_nt_acc(p["a"], sfa, p["b"], sfb, d, c=d)
+    op()
+    g = EventGraph([op] * 4)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(g.durations_ms())
+    g.close()
+    fl = gemm_flops(M, N, K)
+    by = M * K + N * K + 8 * M * N + 4 * M * kp_of(K) + 4 * (N // 128) * kp_of(K)
+    out[f"dense_acc_f32_inplace_{M}x{N}x{K}"] = {"us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
+                                                 "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor"}
+    del p, sfa, sfb, d
+
     # BF16 masked decode (same shapes and masked_m draws, plain bf16 operands)
     def masked_bf16_case(name, q, rng):
         G, max_m, N, K = q["G"], q["max_m"], q["N"], q["K"]

@@ -159,6 +159,23 @@ DG_API dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, c
                       void* d, int M, int N, int K, void* stream);
 
 /*
+ * Dense FP8 NT GEMM with an accumulation matrix, D = C + A . B^T ("DeepInside
+ * DeepGEMM", section 4: the standard non-grouped FP8 NT GEMM computes
+ * D = C + A @ B.T and takes the output dtype).
+ *   a, sfa, b, sfb : as fp8_gemm_nt
+ *   c       : device, [M, N] in D's type (bf16, or fp32 when out_f32 = 1), or
+ *             NULL for C = 0. It is added to the fp32 accumulation before the
+ *             final conversion. c may equal d (in-place accumulation); it must
+ *             not overlap d otherwise. 16-byte aligned.
+ *   d       : device, bf16 [M, N] (out_f32 = 0, round to nearest even) or
+ *             fp32 [M, N] (out_f32 = 1); written completely.
+ * Limits and errors as fp8_gemm_nt; out_f32 outside {0, 1} returns
+ * DG_ERR_INVALID_ARG. Same tiling, split-K and capture safety.
+ */
+DG_API dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c,
+                                 void* d, int M, int N, int K, int out_f32, void* stream);
+
+/*
  * fp8_gemm_nt_noalloc: the dense GEMM of fp8_gemm_nt (same arguments, layouts,
  * limits and results) that allocates no device memory, on any call. The pages
  * of the method have no counterpart of this call; it exists for callers that

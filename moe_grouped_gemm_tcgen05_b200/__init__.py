@@ -24,7 +24,7 @@ __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
-    "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked",
+    "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -87,6 +87,8 @@ def load():
         L.fp8_gemm_nt.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
         L.m_grouped_bf16_gemm_nt_masked.restype = i32
         L.m_grouped_bf16_gemm_nt_masked.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.fp8_gemm_nt_acc.restype = i32
+        L.fp8_gemm_nt_acc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.fp8_gemm_nt_noalloc.restype = i32
         L.fp8_gemm_nt_noalloc.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_contiguous.restype = i32
@@ -185,6 +187,25 @@ def fp8_gemm_nt(a, sfa, b, sfb, d):
     _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
     _need(d, "d", _BF16, (M, N))
     _check("fp8_gemm_nt", load().fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def fp8_gemm_nt_acc(a, sfa, b, sfb, d, c=None):
+    """d[M, N] = c + (a . sfa) @ (b . sfb)^T; d is bf16 or fp32, c (optional) has d's
+    dtype and may be d itself (in-place accumulation)."""
+    _need(a, "a", _FP8)
+    M, K = a.shape
+    _need(b, "b", _FP8)
+    N = b.shape[0]
+    _need(b, "b", _FP8, (N, K))
+    _need(sfa, "sfa", _I32, (M, _kp(K)))
+    _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", (torch.bfloat16, torch.float32), (M, N))
+    if c is not None:
+        _need(c, "c", (d.dtype,), (M, N))
+    _check("fp8_gemm_nt_acc", load().fp8_gemm_nt_acc(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb),
+                                                     None if c is None else _ptr(c), _ptr(d), M, N, K,
+                                                     1 if d.dtype == torch.float32 else 0, _stream()))
     return d
 
 

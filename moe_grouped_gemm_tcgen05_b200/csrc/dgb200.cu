@@ -600,6 +600,34 @@ dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const in
                        static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
 }
 
+dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
+                          int M, int N, int K, int out_f32, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M <= 0 || (out_f32 != 0 && out_f32 != 1)) return DG_ERR_INVALID_ARG;
+    if (c != nullptr && !aligned(c, 16)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);  // bf16 output (the D tensor map covers it either way)
+    p.d32 = out_f32 ? static_cast<float*>(d) : nullptr;
+    p.out_f32 = out_f32;
+    p.c = c;
+    p.meta = nullptr;
+    p.rows = M;
+    p.n = N;
+    p.k = K;
+    p.groups = 1;
+    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
+    const long long esz = out_f32 ? 4 : 2;
+    const long long bytes = (static_cast<long long>(M) + N) * K + esz * M * N * (c != nullptr ? 2 : 1);
+    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
+                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+}
+
 dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
                               int N, int K, int splits, void* stream) {
     dg_status s = check_common(a, sfa, b, sfb, d, N, K);

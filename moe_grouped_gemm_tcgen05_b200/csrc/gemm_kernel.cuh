@@ -110,6 +110,12 @@ struct GemmParams {
     int splits;               // 1 = no split; range i covers K groups [i*G/splits, (i+1)*G/splits)
     float* ws;                // partials: [tile][split][4 row quarters][BN/4][32 lanes][4]
     uint32_t* counters;       // finished units per output tile; zero between calls
+    // dense form: D = C + A.B^T. C (optional, [rows, n] in D's type) is added to
+    // the fp32 accumulation before the final conversion; D is bf16 (d, TMA
+    // stores) or fp32 (d32, direct stores)
+    const void* c;
+    float* d32;
+    int out_f32;
 };
 
 // SCHED_INTS: 32-bit words of shared memory for the tile scheduler (masked:
@@ -867,10 +873,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             auto emit32 = [&](const uint32_t* v, int hc) {
                 const int col = n0 + hc;
                 if (col >= p.n) return;  // warp-uniform: N tail
+                float f[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                if constexpr (KIND == kDense) {
+                    if (p.c != nullptr && valid) {
+                        // + C (N % 8 == 0: whole 8-column pieces are in or out)
+                        const size_t at = out_row * static_cast<size_t>(p.n) + col;
+                        if (p.out_f32) {
+                            const float* crow = static_cast<const float*>(p.c) + at;
+#pragma unroll
+                            for (int q8 = 0; q8 < 4; ++q8) {
+                                if (col + 8 * q8 >= p.n) continue;
+                                const float4 x0 = *reinterpret_cast<const float4*>(crow + 8 * q8);
+                                const float4 x1 = *reinterpret_cast<const float4*>(crow + 8 * q8 + 4);
+                                f[8 * q8] += x0.x; f[8 * q8 + 1] += x0.y; f[8 * q8 + 2] += x0.z; f[8 * q8 + 3] += x0.w;
+                                f[8 * q8 + 4] += x1.x; f[8 * q8 + 5] += x1.y; f[8 * q8 + 6] += x1.z; f[8 * q8 + 7] += x1.w;
+                            }
+                        } else {
+                            const __nv_bfloat16* crow = static_cast<const __nv_bfloat16*>(p.c) + at;
+#pragma unroll
+                            for (int q8 = 0; q8 < 4; ++q8) {
+                                if (col + 8 * q8 >= p.n) continue;
+                                const uint4 x = *reinterpret_cast<const uint4*>(crow + 8 * q8);
+                                const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                                for (int h2 = 0; h2 < 4; ++h2) {
+                                    const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                                    f[8 * q8 + 2 * h2] += c2.x;
+                                    f[8 * q8 + 2 * h2 + 1] += c2.y;
+                                }
+                            }
+                        }
+                    }
+                    if (p.out_f32) {
+                        if (valid) {
+                            float* drow32 = p.d32 + out_row * static_cast<size_t>(p.n) + col;
+#pragma unroll
+                            for (int q4 = 0; q4 < 8; ++q4)
+                                if (col + 4 * q4 < p.n)
+                                    *reinterpret_cast<float4*>(drow32 + 4 * q4) =
+                                        make_float4(f[4 * q4], f[4 * q4 + 1], f[4 * q4 + 2], f[4 * q4 + 3]);
+                        }
+                        return;
+                    }
+                }
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
                     w[i] = *reinterpret_cast<uint32_t*>(&b2);
                 }
                 if (use_tma) {
