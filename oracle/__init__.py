@@ -12,6 +12,7 @@ Modules
 -------
 fp8    -- the OCP E4M3 value table (``e4m3_to_f64``)
 bf16   -- bf16 operand values (``bf16_to_f64``)
+quant  -- the per-token FP8 quantiser with UE8M0 block scales
 ue8m0  -- UE8M0 scale bytes: decode, the capture-safe pack of fp32 scales
           into four bytes per int32, the matching unpack, and the optional
           eager validator
@@ -30,6 +31,7 @@ Every function names the section it follows.
 
 from .fp8 import e4m3_to_f64, E4M3_MAX  # noqa: F401
 from .bf16 import bf16_to_f64  # noqa: F401
+from .quant import e4m3_encode_rne, scale_exponent, quantize_fp8_1x128  # noqa: F401
 from .ue8m0 import (  # noqa: F401
     ue8m0_to_f64,
     pack_ue8m0,

@@ -501,3 +501,90 @@ def test_acc_one_hot_plus_c_exact():
     bv = torch_e4m3(b)
     for m in range(M):
         assert np.array_equal(got[m], c[m] + bv[:, ks[m]])
+
+
+# ------------------------------------------------ per-token quantiser ----
+
+def test_e4m3_encode_round_trips_every_finite_code():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = oracle.e4m3_to_f64(codes)
+    got = oracle.e4m3_encode_rne(vals)
+    # +0 and -0 keep their sign; every other value maps back to its own code
+    assert np.array_equal(got, codes)
+
+
+def test_e4m3_encode_ties_go_to_the_even_code():
+    pos = oracle.e4m3_to_f64(np.arange(127, dtype=np.uint8))
+    mids = (pos[:-1] + pos[1:]) / 2          # exact in float64
+    got = oracle.e4m3_encode_rne(mids)
+    lo = np.arange(126)
+    want = np.where(lo % 2 == 0, lo, lo + 1)
+    assert np.array_equal(got, want.astype(np.uint8))
+    assert np.array_equal(oracle.e4m3_encode_rne(-mids), (want | 0x80).astype(np.uint8))
+
+
+def test_e4m3_encode_matches_torch_float8_cast():
+    rng = np.random.default_rng(31)
+    v = np.concatenate([rng.standard_normal(20000) * 50, rng.standard_normal(5000) * 0.01,
+                        rng.uniform(-448, 448, 5000)]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode_rne(v.astype(np.float64)), ref)
+
+
+def test_scale_exponent_brackets_amax():
+    rng = np.random.default_rng(32)
+    amax = np.concatenate([
+        np.abs(rng.standard_normal(5000)).astype(np.float32),
+        (448.0 * np.ldexp(1.0, rng.integers(-30, 30, 200))).astype(np.float32),         # exactly 448 * 2^k
+        np.nextafter((448.0 * np.ldexp(1.0, rng.integers(-30, 30, 200))).astype(np.float32),
+                     np.float32(np.inf)),                                               # just above
+        np.array([0.0, 1e-9, 9.99e-5], dtype=np.float32)])                              # below the floor
+    e = oracle.scale_exponent(amax)
+    a = np.maximum(amax.astype(np.float64), float(np.float32(1e-4)))
+    assert (448.0 * np.ldexp(1.0, e) >= a).all()
+    assert (448.0 * np.ldexp(1.0, e - 1) < a).all()
+
+
+def test_quantiser_matches_the_input_generator():
+    # two independent routes to the same recipe: the oracle (exact integer
+    # exponent, its own E4M3 encoder) and the input generator (float64 ratio,
+    # torch's float8 cast)
+    from moe_grouped_gemm_tcgen05_b200 import workloads as W
+    rng = np.random.default_rng(33)
+    x = (rng.standard_normal((37, 640)) * rng.uniform(0.01, 100, size=(37, 1))).astype(np.float32)
+    q_ref, sf_ref = W.quantise_rows(x)
+    q, packed, sf = oracle.quantize_fp8_1x128(x.astype(np.float64))
+    assert np.array_equal(q, q_ref)
+    assert np.array_equal(sf, sf_ref)
+    assert np.array_equal(packed, oracle.pack_ue8m0(sf_ref))
+
+
+def _planted_quant(kind):
+    """A copy of the quantiser's exponent rule / encoder with one mistake (CPU only)."""
+    def scale_exp(amax):
+        a = np.maximum(np.asarray(amax, dtype=np.float64), float(np.float32(1e-4)))
+        m2, e2 = np.frexp(a)
+        E, m = e2 - 1, 2.0 * m2
+        if kind == "threshold_inclusive":
+            return (E - 8 + (m >= 1.75)).astype(np.int64)
+        if kind == "floor_not_ceil":
+            return (E - 8).astype(np.int64)
+        return (E - 8 + (m > 1.75)).astype(np.int64)
+    return scale_exp
+
+
+@pytest.mark.parametrize("kind", ["threshold_inclusive", "floor_not_ceil"])
+def test_quantiser_pins_catch_planted_mistakes(kind):
+    amax = (448.0 * np.ldexp(1.0, np.arange(-10, 10))).astype(np.float32)
+    amax = np.concatenate([amax, np.nextafter(amax, np.float32(np.inf)), np.float32([3.0, 0.3])])
+    e = _planted_quant(kind)(amax)
+    a = amax.astype(np.float64)
+    ok = (448.0 * np.ldexp(1.0, e) >= a).all() and (448.0 * np.ldexp(1.0, e - 1) < a).all()
+    assert not ok, kind
+
+
+def test_encoder_pin_catches_ties_away_from_zero():
+    pos = oracle.e4m3_to_f64(np.arange(127, dtype=np.uint8))
+    mids = (pos[:-1] + pos[1:]) / 2
+    away = np.arange(1, 127).astype(np.uint8)              # always the upper neighbour
+    assert not np.array_equal(away, oracle.e4m3_encode_rne(mids))
