@@ -405,6 +405,24 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                                  "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor"}
     del p, sfa, sfb, d
 
+    # per-token FP8 quantiser: bf16 activations [4096, 7168] -> E4M3 + packed UE8M0
+    rows, K = 4096, 7168
+    x = torch.randn((rows, K), device=dev).to(torch.bfloat16)
+    qb = torch.empty((rows, K), dtype=torch.uint8, device=dev)
+    sp = torch.empty((rows, kp_of(K)), dtype=torch.int32, device=dev)
+    op = lambda: dg.quantize_fp8_1x128(x, qb, sp)
+    op()
+    g = EventGraph([op] * reps)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(g.durations_ms())
+    g.close()
+    by = rows * K * 2 + rows * K + rows * kp_of(K) * 4
+    out[f"quantize_fp8_1x128_bf16_{rows}x{K}"] = {"us": ms * 1e3, "GB/s": by / ms / 1e6,
+                                                  "roofline_frac": by / (peaks["hbm"] * 1e9) / (ms * 1e-3),
+                                                  "bound": "hbm"}
+    del x, qb, sp
+
     # BF16 masked decode (same shapes and masked_m draws, plain bf16 operands)
     def masked_bf16_case(name, q, rng):
         G, max_m, N, K = q["G"], q["max_m"], q["N"], q["K"]

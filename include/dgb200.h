@@ -284,6 +284,25 @@ DG_API dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int 
  */
 DG_API dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* bad_count, void* stream);
 
+/*
+ * Per-token FP8 quantiser with UE8M0 block scales ("DeepInside DeepGEMM",
+ * section 5 Production Gotchas: the FP8 cast of the activations and the
+ * packing of their scales go in a dedicated kernel before the GEMM). Produces
+ * the A operand of the GEMMs above in one pass.
+ *   x         : device, [rows, K] bf16 (x_f32 = 0) or fp32 (x_f32 = 1)
+ *   q         : device, E4M3 [rows, K] (written completely)
+ *   sf_packed : device, int32 [rows, ceil(K/512)]: the UE8M0 scale of every
+ *               1x128 block, four per word (byte j of word i = block 4i + j,
+ *               unused bytes of the last word zero), as pack_ue8m0 writes them
+ *   sf_f32    : device, fp32 [rows, K/128] (the same scales as floats), or NULL
+ * Per 1x128 block: amax = max(max |x|, 1e-4), scale 2^e with
+ * e = ceil(log2(amax / 448)), codes = E4M3(x / 2^e) rounded to nearest even.
+ * Limits: K % 128 == 0; x and q 16-byte aligned. Values must be finite (NaN or
+ * infinity give unspecified codes). Capture safe; reads nothing back.
+ */
+DG_API dg_status quantize_fp8_1x128(const void* x, int x_f32, void* q, int32_t* sf_packed, float* sf_f32,
+                                    int64_t rows, int K, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

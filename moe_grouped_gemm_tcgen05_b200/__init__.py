@@ -24,7 +24,7 @@ __all__ = [
     "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
-    "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc",
+    "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc", "quantize_fp8_1x128",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -87,6 +87,8 @@ def load():
         L.fp8_gemm_nt.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
         L.m_grouped_bf16_gemm_nt_masked.restype = i32
         L.m_grouped_bf16_gemm_nt_masked.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.quantize_fp8_1x128.restype = i32
+        L.quantize_fp8_1x128.argtypes = [vp, i32, vp, vp, vp, ctypes.c_int64, i32, vp]
         L.fp8_gemm_nt_acc.restype = i32
         L.fp8_gemm_nt_acc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.fp8_gemm_nt_noalloc.restype = i32
@@ -296,6 +298,25 @@ def pack_ue8m0(sf, out=None):
     _need(out, "out", _I32, (*sf.shape[:-1], kp))
     _check("pack_ue8m0", load().pack_ue8m0(_ptr(sf), _ptr(out), rows, cols, _stream()))
     return out
+
+
+def quantize_fp8_1x128(x, q=None, sf_packed=None, sf_f32=None):
+    """x [rows, K] bf16/fp32 -> (q E4M3 as uint8 [rows, K], packed UE8M0 scales
+    int32 [rows, ceil(K/512)], fp32 scales [rows, K/128] or None)."""
+    _need(x, "x", (torch.bfloat16, torch.float32))
+    rows, K = x.shape
+    if q is None:
+        q = torch.empty((rows, K), dtype=torch.uint8, device=x.device)
+    if sf_packed is None:
+        sf_packed = torch.empty((rows, _kp(K)), dtype=torch.int32, device=x.device)
+    _need(q, "q", _FP8, (rows, K))
+    _need(sf_packed, "sf_packed", _I32, (rows, _kp(K)))
+    if sf_f32 is not None:
+        _need(sf_f32, "sf_f32", (torch.float32,), (rows, K // BLOCK))
+    _check("quantize_fp8_1x128",
+           load().quantize_fp8_1x128(_ptr(x), 1 if x.dtype == torch.float32 else 0, _ptr(q), _ptr(sf_packed),
+                                     None if sf_f32 is None else _ptr(sf_f32), rows, K, _stream()))
+    return q, sf_packed, sf_f32
 
 
 def pack_ue8m0_validate(sf, bad_count):

@@ -780,6 +780,32 @@ dg_status pack_ue8m0(const float* sf, int32_t* packed, int64_t rows, int cols, v
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
 
+dg_status quantize_fp8_1x128(const void* x, int x_f32, void* q, int32_t* sf_packed, float* sf_f32, int64_t rows, int K,
+                             void* stream) {
+    if (!x || !q || !sf_packed || rows <= 0 || K <= 0 || (x_f32 != 0 && x_f32 != 1)) return DG_ERR_INVALID_ARG;
+    if (K % 128 != 0) return DG_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(q, 16) || !aligned(sf_packed, 4) || (sf_f32 && !aligned(sf_f32, 4)))
+        return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    dg_status s = current_device(&st);
+    if (s != DG_OK) return s;
+    const int kb = K / 128;
+    const int kp = (kb + 3) / 4;
+    const int threads = 256;
+    const int64_t warps_needed = (rows * kb + dg::QUANT_UNROLL - 1) / dg::QUANT_UNROLL;
+    int64_t blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
+    const int64_t cap = static_cast<int64_t>(st->sms) * 8;
+    if (blocks > cap) blocks = cap;
+    cudaLaunchAttribute attr[1];
+    const cudaLaunchConfig_t cfg = small_launch(static_cast<unsigned>(blocks), threads, stream, attr);
+    uint32_t* qw = static_cast<uint32_t*>(q);
+    uint8_t* sb = reinterpret_cast<uint8_t*>(sf_packed);
+    const cudaError_t err =
+        x_f32 ? cudaLaunchKernelEx(&cfg, dg::quantize_fp8_1x128_kernel<true>, x, qw, sb, sf_f32, rows, kb, kp)
+              : cudaLaunchKernelEx(&cfg, dg::quantize_fp8_1x128_kernel<false>, x, qw, sb, sf_f32, rows, kb, kp);
+    return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
+}
+
 dg_status pack_ue8m0_validate(const float* sf, int64_t rows, int cols, int32_t* bad_count, void* stream) {
     if (!sf || !bad_count || rows <= 0 || cols <= 0) return DG_ERR_INVALID_ARG;
     if (!aligned(sf, 4) || !aligned(bad_count, 4)) return DG_ERR_ALIGNMENT;
