@@ -791,10 +791,10 @@ dg_status quantize_fp8_1x128(const void* x, int x_f32, void* q, int32_t* sf_pack
     if (s != DG_OK) return s;
     const int kb = K / 128;
     const int kp = (kb + 3) / 4;
-    const int threads = 256;
+    const int threads = dg::QUANT_THREADS;
     const int64_t warps_needed = (rows * kb + dg::QUANT_UNROLL - 1) / dg::QUANT_UNROLL;
     int64_t blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
-    const int64_t cap = static_cast<int64_t>(st->sms) * 8;
+    const int64_t cap = static_cast<int64_t>(st->sms) * dg::QUANT_BLOCKS_PER_SM;
     if (blocks > cap) blocks = cap;
     cudaLaunchAttribute attr[1];
     const cudaLaunchConfig_t cfg = small_launch(static_cast<unsigned>(blocks), threads, stream, attr);
