@@ -42,6 +42,7 @@ from .gemm import (  # noqa: F401
     dequant_rows,
     dequant_weights,
     fp8_gemm_nt,
+    fp8_gemm,
     fp8_gemm_nt_acc,
     fp8_gemm_nt_sampled,
     fp8_gemm_nt_points,

@@ -181,6 +181,26 @@ def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb) -> np.ndarray:
     return np.einsum("ik,ik->i", A, B)
 
 
+# ---- dense GEMM with other operand layouts --------------------------------------
+
+def fp8_gemm(a, sfa, b, sfb, layout: str) -> np.ndarray:
+    """Dense FP8 GEMM D[m, n] = sum_k A^[m, k] B^[n, k] for the operand layouts
+    that "DeepInside DeepGEMM" §2 lists for SM100 (NT, TN, NN, TT). The first
+    letter is A's storage: "n" = [M, K] (K contiguous), "t" = [K, M]; the second
+    is B's: "t" = [N, K] (K contiguous), "n" = [K, N]. The scales do not depend
+    on the storage: sfa is [M, KP] (one per row and 128-K block), sfb is
+    [ceil(N/128), KP]. Reading: the letters follow the NT GEMM of §4 (A as
+    given, B transposed); the pages name the layouts without defining them."""
+    layout = layout.lower()
+    if layout not in ("nt", "tn", "nn", "tt"):
+        raise ValueError(f"unknown layout {layout!r}")
+    A = np.asarray(a, dtype=np.uint8)
+    B = np.asarray(b, dtype=np.uint8)
+    A_mk = A if layout[0] == "n" else A.T
+    B_nk = B if layout[1] == "t" else B.T
+    return fp8_gemm_nt(np.ascontiguousarray(A_mk), sfa, np.ascontiguousarray(B_nk), sfb)
+
+
 # ---- dense GEMM with an accumulation matrix ------------------------------------
 
 def fp8_gemm_nt_acc(a, sfa, b, sfb, c=None) -> np.ndarray:

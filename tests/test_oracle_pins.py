@@ -588,3 +588,39 @@ def test_encoder_pin_catches_ties_away_from_zero():
     mids = (pos[:-1] + pos[1:]) / 2
     away = np.arange(1, 127).astype(np.uint8)              # always the upper neighbour
     assert not np.array_equal(away, oracle.e4m3_encode_rne(mids))
+
+
+# ------------------------------------------- other operand layouts ----
+
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_layouts_equal_exact_rational_brute_force(layout):
+    # D[m, n] = sum_k A[m, k] B[n, k] with each operand read from its own
+    # storage order, computed with exact rationals straight from the codes
+    rng = np.random.default_rng(41)
+    M, N, K = 3, 5, 256
+    a_mk = _rand_codes(rng, (M, K))
+    b_nk = _rand_codes(rng, (N, K))
+    ea = rng.integers(120, 135, size=(M, 2)).astype(np.uint8)
+    eb = rng.integers(120, 135, size=(1, 2)).astype(np.uint8)
+    a = a_mk if layout[0] == "n" else np.ascontiguousarray(a_mk.T)
+    b = b_nk if layout[1] == "t" else np.ascontiguousarray(b_nk.T)
+    got = oracle.fp8_gemm(a, _pack_bytes(ea), b, _pack_bytes(eb), layout)
+    av, bv = torch_e4m3(a), torch_e4m3(b)
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                x = av[m, k] if layout[0] == "n" else av[k, m]
+                y = bv[n, k] if layout[1] == "t" else bv[k, n]
+                acc += (Fraction(float(x)) * Fraction(2) ** (int(ea[m, k // 128]) - 127) *
+                        Fraction(float(y)) * Fraction(2) ** (int(eb[0, k // 128]) - 127))
+            assert Fraction(got[m, n]) == acc, (layout, m, n)
+
+
+def test_layout_pin_catches_an_unswapped_operand():
+    rng = np.random.default_rng(42)
+    M, K = 128, 128
+    a = _rand_codes(rng, (M, K))
+    ones = _pack_bytes(np.full((M, 1), 127, np.uint8))
+    # reading a [K, M] A as if it were [M, K] changes the result
+    assert not np.array_equal(oracle.fp8_gemm(a, ones, a, ones, "tt"), oracle.fp8_gemm(a, ones, a, ones, "nt"))
