@@ -405,6 +405,28 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                                  "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor"}
     del p, sfa, sfb, d
 
+    # other operand layouts (A stored [K, M] and/or B stored [K, N]), 4096x7168x16384
+    M, N, K = 4096, 7168, 16384
+    p = W.workload1_t(M, N, K, dev)
+    sfa, sfb = dg.pack_ue8m0(p["sfa_f32"]), dg.pack_ue8m0(p["sfb_f32"])
+    d = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    a_km = p["a"].t().contiguous()
+    b_kn = p["b"].t().contiguous()
+    for name, fn, a_op, b_op in (("nn", dg.fp8_gemm_nn, p["a"], b_kn), ("tn", dg.fp8_gemm_tn, a_km, b_kn),
+                                 ("tt", dg.fp8_gemm_tt, a_km, p["b"])):
+        op = lambda fn=fn, a_op=a_op, b_op=b_op: fn(a_op, sfa, b_op, sfb, d)
+        op()
+        g = EventGraph([op] * 4)
+        g.replay()
+        torch.cuda.synchronize()
+        ms = statistics.median(g.durations_ms())
+        g.close()
+        fl = gemm_flops(M, N, K)
+        out[f"dense_{name}_{M}x{N}x{K}"] = {"us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
+                                            "roofline_frac": frac_tensor_mem(fl, dense_bytes(M, N, K), ms),
+                                            "bound": "tensor"}
+    del p, sfa, sfb, d, a_km, b_kn
+
     # per-token FP8 quantiser: bf16 activations [4096, 7168] -> E4M3 + packed UE8M0
     rows, K = 4096, 7168
     x = torch.randn((rows, K), device=dev).to(torch.bfloat16)

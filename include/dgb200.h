@@ -159,6 +159,28 @@ DG_API dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, c
                       void* d, int M, int N, int K, void* stream);
 
 /*
+ * Dense FP8 GEMM in the other operand layouts ("DeepInside DeepGEMM", section 2:
+ * SM100 supports the NT, TN, NN and TT layouts). D[m, n] = sum_k A[m, k] B[n, k]
+ * with scales as in fp8_gemm_nt (sfa [M, KP] by rows of A, sfb [ceil(N/128), KP]
+ * by 128-row blocks of B), whatever the storage:
+ *   fp8_gemm_nn : a E4M3 [M, K] (K contiguous), b E4M3 [K, N] (N contiguous)
+ *   fp8_gemm_tn : a E4M3 [K, M] (M contiguous), b E4M3 [K, N] (N contiguous)
+ *   fp8_gemm_tt : a E4M3 [K, M] (M contiguous), b E4M3 [N, K] (K contiguous)
+ *   d           : bf16 [M, N]
+ * An operand stored M- or N-contiguous is loaded in 128-byte swizzle atoms of
+ * that dimension and fed to the MMA as an MN-major operand (no transposition
+ * pass). Limits as fp8_gemm_nt, plus M % 16 == 0 when A is stored [K, M] and
+ * N % 16 == 0 when B is stored [K, N] (16-byte row pitch). Single CTAs, no
+ * split-K; N tile 128 or 256.
+ */
+DG_API dg_status fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                             int N, int K, void* stream);
+DG_API dg_status fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                             int N, int K, void* stream);
+DG_API dg_status fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                             int N, int K, void* stream);
+
+/*
  * Dense FP8 NT GEMM with an accumulation matrix, D = C + A . B^T ("DeepInside
  * DeepGEMM", section 4: the standard non-grouped FP8 NT GEMM computes
  * D = C + A @ B.T and takes the output dtype).

@@ -25,6 +25,7 @@ __all__ = [
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
     "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc", "quantize_fp8_1x128",
+    "fp8_gemm_nn", "fp8_gemm_tn", "fp8_gemm_tt",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -89,6 +90,9 @@ def load():
         L.m_grouped_bf16_gemm_nt_masked.argtypes = [vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.quantize_fp8_1x128.restype = i32
         L.quantize_fp8_1x128.argtypes = [vp, i32, vp, vp, vp, ctypes.c_int64, i32, vp]
+        for name in ("fp8_gemm_nn", "fp8_gemm_tn", "fp8_gemm_tt"):
+            getattr(L, name).restype = i32
+            getattr(L, name).argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp]
         L.fp8_gemm_nt_acc.restype = i32
         L.fp8_gemm_nt_acc.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.fp8_gemm_nt_noalloc.restype = i32
@@ -190,6 +194,38 @@ def fp8_gemm_nt(a, sfa, b, sfb, d):
     _need(d, "d", _BF16, (M, N))
     _check("fp8_gemm_nt", load().fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
     return d
+
+
+def _fp8_gemm_layout(name, a, sfa, b, sfb, d, a_mk: bool, b_nk: bool):
+    _need(a, "a", _FP8)
+    _need(b, "b", _FP8)
+    if a_mk:
+        M, K = a.shape
+    else:
+        K, M = a.shape
+    N = b.shape[0] if b_nk else b.shape[1]
+    _need(a, "a", _FP8, (M, K) if a_mk else (K, M))
+    _need(b, "b", _FP8, (N, K) if b_nk else (K, N))
+    _need(sfa, "sfa", _I32, (M, _kp(K)))
+    _need(sfb, "sfb", _I32, ((N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (M, N))
+    _check(name, getattr(load(), name)(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def fp8_gemm_nn(a, sfa, b, sfb, d):
+    """d[M, N] = (a . sfa) @ (b . sfb) for E4M3 a [M, K], b [K, N]."""
+    return _fp8_gemm_layout("fp8_gemm_nn", a, sfa, b, sfb, d, True, False)
+
+
+def fp8_gemm_tn(a, sfa, b, sfb, d):
+    """d[M, N] = (a . sfa)^T @ (b . sfb) for E4M3 a [K, M], b [K, N]."""
+    return _fp8_gemm_layout("fp8_gemm_tn", a, sfa, b, sfb, d, False, False)
+
+
+def fp8_gemm_tt(a, sfa, b, sfb, d):
+    """d[M, N] = (a . sfa)^T @ (b . sfb)^T for E4M3 a [K, M], b [N, K]."""
+    return _fp8_gemm_layout("fp8_gemm_tt", a, sfa, b, sfb, d, False, True)
 
 
 def fp8_gemm_nt_acc(a, sfa, b, sfb, d, c=None):

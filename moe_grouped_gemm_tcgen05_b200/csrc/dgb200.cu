@@ -91,9 +91,9 @@ const int g_k_rotate = [] {
 
 // --------------------------------------------------------------- kernels ----
 
-template <int BN, int KIND, int CG, int DT>
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0>
 void* kernel_ptr() {
-    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT>);
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT, LAYOUT>);
 }
 
 struct KernelEntry {
@@ -101,14 +101,17 @@ struct KernelEntry {
     int kind;
     int cg;      // CTAs per MMA unit (1, or a cluster pair)
     int dt;      // operand type (dg::kE4M3 block-scaled, dg::kBF16)
+    int layout;  // dense: bit 0 A stored [K, M], bit 1 B stored [K, N]
     void* fn;
     int smem;
     int stages;  // depth of the operand ring
 };
 
-#define DG_ENTRY_T(BN, KIND, CG, DT)                                                                            \
-    {BN, KIND, CG, DT, kernel_ptr<BN, KIND, CG, DT>(),                                                          \
+#define DG_ENTRY_TL(BN, KIND, CG, DT, LAYOUT)                                                                   \
+    {BN, KIND, CG, DT, LAYOUT, kernel_ptr<BN, KIND, CG, DT, LAYOUT>(),                                          \
      dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES}
+#define DG_ENTRY_T(BN, KIND, CG, DT) DG_ENTRY_TL(BN, KIND, CG, DT, 0)
+#define DG_LAYOUT(BN, LAYOUT) DG_ENTRY_TL(BN, dg::kDense, 1, dg::kE4M3, LAYOUT)
 #define DG_ENTRY(BN, KIND, CG) DG_ENTRY_T(BN, KIND, CG, dg::kE4M3)
 #define DG_BF16_MASKED(BN) DG_ENTRY_T(BN, dg::kMasked, 1, dg::kBF16)
 #define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1)
@@ -122,6 +125,7 @@ const KernelEntry kKernels[] = {
     DG_ENTRY(224, dg::kContiguous, 2), DG_ENTRY(256, dg::kContiguous, 2),
     DG_BF16_MASKED(64), DG_BF16_MASKED(96), DG_BF16_MASKED(128), DG_BF16_MASKED(160),
     DG_BF16_MASKED(192), DG_BF16_MASKED(224), DG_BF16_MASKED(256),
+    DG_LAYOUT(128, 1), DG_LAYOUT(256, 1), DG_LAYOUT(128, 2), DG_LAYOUT(256, 2), DG_LAYOUT(128, 3), DG_LAYOUT(256, 3),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
@@ -251,6 +255,19 @@ bool encode_kmajor(CUtensorMap* map, const void* base, int rank, uint64_t k, uin
     return r == CUDA_SUCCESS;
 }
 
+// MN-major E4M3 operand stored [K, mn] (mn contiguous): boxes of 128 bytes of
+// mn by 128 K rows with the 128-byte swizzle.
+bool encode_mnmajor(CUtensorMap* map, const void* base, uint64_t mn, uint64_t k) {
+    cuuint64_t dims[2] = {mn, k};
+    cuuint64_t strides[1] = {mn};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t elem[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // bf16 output, written by TMA in 32x32 boxes with the 64-byte swizzle.
 bool encode_d_bf16(CUtensorMap* map, void* base, int rank, uint64_t n, uint64_t rows, uint64_t mats) {
     cuuint64_t dims[3] = {n, rows, mats};
@@ -324,7 +341,8 @@ struct SplitScratch {
 };
 
 TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                          long long unique_bytes, int forced_splits, const SplitScratch& scratch, int dt = dg::kE4M3) {
+                          long long unique_bytes, int forced_splits, const SplitScratch& scratch, int dt = dg::kE4M3,
+                          int layout = 0) {
     const int kb = k / (dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K (one pipeline stage each)
     const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
@@ -334,7 +352,7 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
-        if (e.kind != kind || e.dt != dt) continue;
+        if (e.kind != kind || e.dt != dt || e.layout != layout) continue;
         if (forced_bn != 0 && e.bn != forced_bn) continue;
         if (forced_cg != 0 && e.cg != forced_cg) continue;
         if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
@@ -393,10 +411,10 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
 // The library's own choice: the allocated split-K workspace, and the split
 // count forced by dgb200_set_splits (dense form).
 TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                       long long unique_bytes, int dt = dg::kE4M3) {
+                       long long unique_bytes, int dt = dg::kE4M3, int layout = 0) {
     const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
     const SplitScratch scratch{st->split_ws != nullptr, static_cast<double>(kSplitWsBytes), kSplitCounters};
-    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt);
+    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt, layout);
 }
 
 // Bytes of split-K partials a choice writes (0 when it does not split).
@@ -458,11 +476,17 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.ws = choice.splits > 1 ? ws : nullptr;
     p.counters = choice.splits > 1 ? counters : nullptr;
     p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
-    if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128, e->dt))
+    if (e->layout & 1) {
+        if (!encode_mnmajor(&p.tma_a, a, a_rows, static_cast<uint64_t>(p.k))) return DG_ERR_INVALID_ARG;
+    } else if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128, e->dt)) {
         return DG_ERR_INVALID_ARG;
-    if (!encode_kmajor(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats, static_cast<uint32_t>(bn / cg),
-                       e->dt))
+    }
+    if (e->layout & 2) {
+        if (!encode_mnmajor(&p.tma_b, b, b_rows, static_cast<uint64_t>(p.k))) return DG_ERR_INVALID_ARG;
+    } else if (!encode_kmajor(&p.tma_b, b, b_rank, static_cast<uint64_t>(p.k), b_rows, b_mats,
+                              static_cast<uint32_t>(bn / cg), e->dt)) {
         return DG_ERR_INVALID_ARG;
+    }
     if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
     // contiguous pairs walk two passes (see next_tile in gemm_kernel.cuh)
     const long long tiles = (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks) *
@@ -502,8 +526,9 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
                       long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
                       int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats,
-                      int dt = dg::kE4M3) {
-    const TileChoice choice = choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt);
+                      int dt = dg::kE4M3, int layout = 0) {
+    const TileChoice choice =
+        choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt, layout);
     return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
                             a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
 }
@@ -598,6 +623,46 @@ dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const in
     const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
     return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
                        static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+}
+
+// Dense GEMM in the TN/NN/TT layouts (layout bit 0: A stored [K, M]; bit 1: B
+// stored [K, N]).
+dg_status fp8_gemm_layout(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
+                          int K, int layout, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M <= 0) return DG_ERR_INVALID_ARG;
+    if (((layout & 1) && M % 16 != 0) || ((layout & 2) && N % 16 != 0)) return DG_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.rows = M;
+    p.n = N;
+    p.k = K;
+    p.groups = 1;
+    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
+    const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
+    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
+                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1, dg::kE4M3, layout);
+}
+
+dg_status fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
+                      int K, void* stream) {
+    return fp8_gemm_layout(a, sfa, b, sfb, d, M, N, K, 2, stream);
+}
+
+dg_status fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
+                      int K, void* stream) {
+    return fp8_gemm_layout(a, sfa, b, sfb, d, M, N, K, 3, stream);
+}
+
+dg_status fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
+                      int K, void* stream) {
+    return fp8_gemm_layout(a, sfa, b, sfb, d, M, N, K, 1, stream);
 }
 
 dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,

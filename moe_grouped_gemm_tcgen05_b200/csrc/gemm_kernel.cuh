@@ -394,11 +394,31 @@ struct ScaleWords {
 
 // ------------------------------------------------------------------ kernel --
 
-template <int BN, int KIND, int CG, int DT>
+// LAYOUT bit 0: A is stored MN-major ([K, M], M contiguous); bit 1: B is
+// stored MN-major ([K, N]). MN-major tiles are loaded as 128-byte swizzle
+// atoms of M or N by K rows and described to the MMA as such.
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
     static_assert(CG == 1 || KIND != kMasked, "CTA pairs are built for the dense and contiguous forms");
     static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
+    static_assert(LAYOUT == 0 || (KIND == kDense && CG == 1 && DT == kE4M3), "layouts: dense, single CTAs");
+    static_assert(!(LAYOUT & 2) || BN % 128 == 0, "an MN-major B tile is whole 128-byte atoms");
+    constexpr bool kMnA = (LAYOUT & 1) != 0;
+    constexpr bool kMnB = (LAYOUT & 2) != 0;
     using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT>;
+    // instruction descriptor with the operands' major modes
+    constexpr uint32_t kIdesc = Cfg::IDESC | (kMnA ? (1u << 15) : 0u) | (kMnB ? (1u << 16) : 0u);
+    // MN-major descriptor strides: one atom is 128 K-rows x 128 bytes
+    constexpr uint32_t kMnAtomBytes = BK * 128;
+    // Every MMA reads a single atom of an MN-major operand (A tiles are 128
+    // rows; an MN-major B tile is issued one 128-column atom at a time), so the
+    // stride between atoms along MN is never used; both offsets are set to the
+    // 1024-byte stride between groups of 8 K-rows.
+    constexpr uint32_t kMnLbo = 8 * 128;
+    constexpr uint32_t kMnSbo = 8 * 128;
+    constexpr int kBParts = kMnB ? BN / 128 : 1;   // MMAs per K-step along N
+    constexpr uint32_t kIdescPart = kMnB ? (idesc_mxf8_e4m3_ue8m0(BM * CG, 128) | (kMnA ? (1u << 15) : 0u) | (1u << 16))
+                                         : kIdesc;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int NUM_ACC = Cfg::NUM_ACC;
 
@@ -564,10 +584,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
                         if constexpr (KIND == kMasked) {
                             tma_load_3d(a_dst, &p.tma_a, &full_bar[stage], kx, a_row, cur.g);
+                        } else if constexpr (kMnA) {
+                            tma_load_2d(a_dst, &p.tma_a, &full_bar[stage], a_row, kx);   // {M, K} box
                         } else {
                             tma_load_2d(a_dst, &p.tma_a, &full_bar[stage], kx, a_row);
                         }
-                        if constexpr (KIND == kDense) {
+                        if constexpr (kMnB) {
+#pragma unroll
+                            for (int at = 0; at < BN / 128; ++at)                          // {N, K} boxes
+                                tma_load_2d(b_dst + at * kMnAtomBytes, &p.tma_b, &full_bar[stage], b_row + 128 * at, kx);
+                        } else if constexpr (KIND == kDense) {
                             tma_load_2d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row);
                         } else {
                             tma_load_3d(b_dst, &p.tma_b, &full_bar[stage], kx, b_row, g);
@@ -729,20 +755,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         // the tensor core's shared-memory reads: no fence needed here
                         if (!wait_warp(&full_bar[stage], phase, p, s_abort)) { aborted = true; break; }
                         const uint32_t sf_id = static_cast<uint32_t>(kb & 3);
-                        const uint32_t idesc = idesc_with_sf_id(Cfg::IDESC, sf_id);
+                        const uint32_t idesc = idesc_with_sf_id(kIdesc, sf_id);
                         const uint32_t sfa_t = sf_cur | (sf_id << 30);
                         const uint32_t sfb_t = (sf_cur + 4) | (sf_id << 30);
-                        const uint64_t adesc = smem_desc_sw128(smem_u32(smem_a + stage * Cfg::A_BYTES));
-                        const uint64_t bdesc = smem_desc_sw128(smem_u32(smem_b + stage * Cfg::B_BYTES));
+                        const uint64_t adesc =
+                            kMnA ? smem_desc_sw128_mn(smem_u32(smem_a + stage * Cfg::A_BYTES), kMnLbo, kMnSbo)
+                                 : smem_desc_sw128(smem_u32(smem_a + stage * Cfg::A_BYTES));
+                        const uint64_t bdesc =
+                            kMnB ? smem_desc_sw128_mn(smem_u32(smem_b + stage * Cfg::B_BYTES), kMnLbo, kMnSbo)
+                                 : smem_desc_sw128(smem_u32(smem_b + stage * Cfg::B_BYTES));
                         if (elect_one()) {
                             // four MMAs per 128-byte row of K: E4M3 K = 32, BF16 K = 16 per instruction;
                             // each advances the start address by 32 bytes inside the swizzled row
 #pragma unroll
                             for (int k = 0; k < 4; ++k) {
+                                // K-major: the next 32 bytes of K in each swizzled row;
+                                // MN-major: the next 32 K-rows (4 groups of 8 rows of 128 bytes)
                                 const uint64_t koff = static_cast<uint64_t>((k * 32) >> 4);
+                                const uint64_t koff_mn = static_cast<uint64_t>((k * 32 * 128) >> 4);
                                 const uint32_t accumulate = (gi > c.kg0 || kb > kb0 || k > 0) ? 1u : 0u;
-                                if constexpr (DT == kE4M3)
-                                    tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + koff, bdesc + koff, idesc, sfa_t,
+                                if constexpr (DT == kE4M3 && kBParts > 1) {
+                                    // MN-major B: one N = 128 MMA per atom, into its
+                                    // accumulator columns, with its chunk of B scales
+#pragma unroll
+                                    for (int part = 0; part < kBParts; ++part)
+                                        tc_mma_mxf8f6f4_block_scale<CG>(
+                                            d_tmem + 128 * part, adesc + (kMnA ? koff_mn : koff),
+                                            bdesc + ((part * kMnAtomBytes) >> 4) + koff_mn,
+                                            idesc_with_sf_id(kIdescPart, sf_id), sfa_t,
+                                            (sf_cur + 4 + 4 * part) | (sf_id << 30), accumulate);
+                                } else if constexpr (DT == kE4M3)
+                                    tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + (kMnA ? koff_mn : koff),
+                                                                    bdesc + (kMnB ? koff_mn : koff), idesc, sfa_t,
                                                                     sfb_t, accumulate);
                                 else
                                     tc_mma_f16<CG>(d_tmem, adesc + koff, bdesc + koff, Cfg::IDESC, accumulate);

@@ -348,6 +348,20 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory descriptor of an MN-major operand tile with the 128-byte
+// swizzle: rows are K, each holding 128 bytes (one swizzle atom) of the M or N
+// dimension, as a TMA box {128 bytes of MN, K rows} writes it. `lbo` is the byte
+// stride between swizzle atoms along MN, `sbo` between groups of 8 K-rows.
+__device__ __forceinline__ uint64_t smem_desc_sw128_mn(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
 // Descriptor of a 32-row x 16-byte unswizzled matrix (rows contiguous) used as
 // the source of tcgen05.cp 32x128b: four 8x16-byte core matrices 128 B apart.
 __device__ __forceinline__ uint64_t smem_desc_sf(uint32_t saddr) {
