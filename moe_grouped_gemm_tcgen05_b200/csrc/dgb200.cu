@@ -91,9 +91,9 @@ const int g_k_rotate = [] {
 
 // --------------------------------------------------------------- kernels ----
 
-template <int BN, int KIND, int CG, int DT, int LAYOUT = 0>
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0>
 void* kernel_ptr() {
-    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT, LAYOUT>);
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT, LAYOUT, EPI>);
 }
 
 struct KernelEntry {
@@ -102,15 +102,18 @@ struct KernelEntry {
     int cg;      // CTAs per MMA unit (1, or a cluster pair)
     int dt;      // operand type (dg::kE4M3 block-scaled, dg::kBF16)
     int layout;  // dense: bit 0 A stored [K, M], bit 1 B stored [K, N]
+    int epi;     // dense: 1 = epilogue of D = C + A.B^T (bf16 or fp32 D)
     void* fn;
     int smem;
     int stages;  // depth of the operand ring
 };
 
-#define DG_ENTRY_TL(BN, KIND, CG, DT, LAYOUT)                                                                   \
-    {BN, KIND, CG, DT, LAYOUT, kernel_ptr<BN, KIND, CG, DT, LAYOUT>(),                                          \
+#define DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, EPI)                                                             \
+    {BN, KIND, CG, DT, LAYOUT, EPI, kernel_ptr<BN, KIND, CG, DT, LAYOUT, EPI>(),                                \
      dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES}
+#define DG_ENTRY_TL(BN, KIND, CG, DT, LAYOUT) DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, 0)
 #define DG_ENTRY_T(BN, KIND, CG, DT) DG_ENTRY_TL(BN, KIND, CG, DT, 0)
+#define DG_ACC(BN, CG) DG_ENTRY_TLE(BN, dg::kDense, CG, dg::kE4M3, 0, 1)
 #define DG_LAYOUT(BN, LAYOUT) DG_ENTRY_TL(BN, dg::kDense, 1, dg::kE4M3, LAYOUT)
 #define DG_ENTRY(BN, KIND, CG) DG_ENTRY_T(BN, KIND, CG, dg::kE4M3)
 #define DG_BF16_MASKED(BN) DG_ENTRY_T(BN, dg::kMasked, 1, dg::kBF16)
@@ -126,6 +129,8 @@ const KernelEntry kKernels[] = {
     DG_BF16_MASKED(64), DG_BF16_MASKED(96), DG_BF16_MASKED(128), DG_BF16_MASKED(160),
     DG_BF16_MASKED(192), DG_BF16_MASKED(224), DG_BF16_MASKED(256),
     DG_LAYOUT(128, 1), DG_LAYOUT(256, 1), DG_LAYOUT(128, 2), DG_LAYOUT(256, 2), DG_LAYOUT(128, 3), DG_LAYOUT(256, 3),
+    DG_ACC(64, 1), DG_ACC(96, 1), DG_ACC(128, 1), DG_ACC(160, 1), DG_ACC(192, 1), DG_ACC(224, 1), DG_ACC(256, 1),
+    DG_ACC(128, 2), DG_ACC(160, 2), DG_ACC(192, 2), DG_ACC(224, 2), DG_ACC(256, 2),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
@@ -342,7 +347,7 @@ struct SplitScratch {
 
 TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
                           long long unique_bytes, int forced_splits, const SplitScratch& scratch, int dt = dg::kE4M3,
-                          int layout = 0) {
+                          int layout = 0, int epi = 0) {
     const int kb = k / (dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K (one pipeline stage each)
     const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
@@ -352,7 +357,7 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
-        if (e.kind != kind || e.dt != dt || e.layout != layout) continue;
+        if (e.kind != kind || e.dt != dt || e.layout != layout || e.epi != epi) continue;
         if (forced_bn != 0 && e.bn != forced_bn) continue;
         if (forced_cg != 0 && e.cg != forced_cg) continue;
         if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
@@ -411,10 +416,10 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
 // The library's own choice: the allocated split-K workspace, and the split
 // count forced by dgb200_set_splits (dense form).
 TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
-                       long long unique_bytes, int dt = dg::kE4M3, int layout = 0) {
+                       long long unique_bytes, int dt = dg::kE4M3, int layout = 0, int epi = 0) {
     const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
     const SplitScratch scratch{st->split_ws != nullptr, static_cast<double>(kSplitWsBytes), kSplitCounters};
-    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt, layout);
+    return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt, layout, epi);
 }
 
 // Bytes of split-K partials a choice writes (0 when it does not split).
@@ -526,9 +531,9 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
 dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic, long long max_tiles_per_nblock,
                       long long unique_bytes, void* stream, DeviceState* st, const void* a, const void* b, int a_rank,
                       int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows, uint64_t b_mats,
-                      int dt = dg::kE4M3, int layout = 0) {
+                      int dt = dg::kE4M3, int layout = 0, int epi = 0) {
     const TileChoice choice =
-        choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt, layout);
+        choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt, layout, epi);
     return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
                             a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
 }
@@ -690,7 +695,7 @@ dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* b, cons
     const long long esz = out_f32 ? 4 : 2;
     const long long bytes = (static_cast<long long>(M) + N) * K + esz * M * N * (c != nullptr ? 2 : 1);
     return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
-                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1, dg::kE4M3, 0, 1);
 }
 
 dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,

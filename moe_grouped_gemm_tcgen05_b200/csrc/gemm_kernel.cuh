@@ -397,12 +397,15 @@ struct ScaleWords {
 // LAYOUT bit 0: A is stored MN-major ([K, M], M contiguous); bit 1: B is
 // stored MN-major ([K, N]). MN-major tiles are loaded as 128-byte swizzle
 // atoms of M or N by K rows and described to the MMA as such.
-template <int BN, int KIND, int CG, int DT, int LAYOUT = 0>
+// EPI 1: the epilogue of D = C + A.B^T (optional C, bf16 or fp32 D; dense form);
+// EPI 0: plain bf16 D.
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
     static_assert(CG == 1 || KIND != kMasked, "CTA pairs are built for the dense and contiguous forms");
     static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
     static_assert(LAYOUT == 0 || (KIND == kDense && CG == 1 && DT == kE4M3), "layouts: dense, single CTAs");
     static_assert(!(LAYOUT & 2) || BN % 128 == 0, "an MN-major B tile is whole 128-byte atoms");
+    static_assert(EPI == 0 || (KIND == kDense && DT == kE4M3 && LAYOUT == 0), "C / fp32 epilogue: dense NT form");
     constexpr bool kMnA = (LAYOUT & 1) != 0;
     constexpr bool kMnB = (LAYOUT & 2) != 0;
     using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT>;
@@ -920,7 +923,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 float f[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-                if constexpr (KIND == kDense) {
+                if constexpr (EPI == 1) {
                     if (p.c != nullptr && valid) {
                         // + C (N % 8 == 0: whole 8-column pieces are in or out)
                         const size_t at = out_row * static_cast<size_t>(p.n) + col;
