@@ -17,6 +17,12 @@ weights one per 128x128 block. The dequantised operands are
 where ea / eb are the bytes of the packed int32 scale rows (byte j of word i is
 K-block 4*i + j). The reference result is A^ . B^^T in float64.
 
+The same page's minimal FP8 GEMM example gives B one scale row per row of B
+(``b_sf`` of shape [n, k // 128]), i.e. 1x128 blocks for the weights as well.
+Every dense and grouped function below takes ``sfb_gran_n``: the number of
+rows of B that share one scale row, 128 (the 128x128 blocks above, sfb
+[ceil(N/128), KP]) or 1 (sfb [N, KP], B^[n, k] scaled by eb[n, k // 128]).
+
 Grouped forms (readings; the pages name them but print no definition beyond
 the call shape):
 * contiguous: rows of A are concatenated by expert; ``m_indices[r]`` gives the
@@ -57,43 +63,53 @@ def dequant_rows(a, sfa) -> np.ndarray:
     return (vals * scale[:, :, None]).reshape(R, K)
 
 
-def dequant_weights(b, sfb, cols=None) -> np.ndarray:
-    """B^ for weight rows: b uint8 [N, K], sfb int32 [ceil(N/128), KP] -> float64.
+def _gran(sfb_gran_n) -> int:
+    if sfb_gran_n not in (1, BLOCK):
+        raise ValueError(f"sfb_gran_n={sfb_gran_n}: B scale rows cover 1 or {BLOCK} rows of B")
+    return int(sfb_gran_n)
+
+
+def dequant_weights(b, sfb, cols=None, sfb_gran_n=BLOCK) -> np.ndarray:
+    """B^ for weight rows: b uint8 [N, K], sfb int32 [ceil(N/gran), KP] -> float64.
 
     ``cols`` (optional) selects which rows n of B to dequantise, so that sampled
-    checks need not expand the whole weight.
+    checks need not expand the whole weight. Row n of B takes scale row
+    n // sfb_gran_n (128x128 blocks for 128, one scale row per row of B for 1).
     """
+    gran = _gran(sfb_gran_n)
     b = np.asarray(b, dtype=np.uint8)
     N, K = b.shape
     KB = _kb(K)
+    if np.asarray(sfb).shape[0] != -(-N // gran):
+        raise ValueError(f"sfb has {np.asarray(sfb).shape[0]} scale rows; N={N} at granularity {gran} needs {-(-N // gran)}")
     n = np.arange(N) if cols is None else np.asarray(cols, dtype=np.int64)
-    block_scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))  # [ceil(N/128), KB]
-    scale = block_scale[n // BLOCK]  # one per 128x128 block
+    row_scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))  # [ceil(N/gran), KB]
+    scale = row_scale[n // gran]
     vals = e4m3_to_f64(b[n]).reshape(len(n), KB, BLOCK)
     return (vals * scale[:, :, None]).reshape(len(n), K)
 
 
-def fp8_gemm_nt(a, sfa, b, sfb) -> np.ndarray:
+def fp8_gemm_nt(a, sfa, b, sfb, sfb_gran_n=BLOCK) -> np.ndarray:
     """Dense D[M, N] = A^ . B^^T in float64."""
-    return dequant_rows(a, sfa) @ dequant_weights(b, sfb).T
+    return dequant_rows(a, sfa) @ dequant_weights(b, sfb, sfb_gran_n=sfb_gran_n).T
 
 
-def fp8_gemm_nt_sampled(a, sfa, b, sfb, rows, cols) -> np.ndarray:
+def fp8_gemm_nt_sampled(a, sfa, b, sfb, rows, cols, sfb_gran_n=BLOCK) -> np.ndarray:
     """D[rows[i], cols[i]] of the dense GEMM, one output at a time (float64)."""
     rows = np.asarray(rows, dtype=np.int64)
     cols = np.asarray(cols, dtype=np.int64)
     ur, ri = np.unique(rows, return_inverse=True)
     uc, ci = np.unique(cols, return_inverse=True)
     ah = dequant_rows(np.asarray(a)[ur], np.asarray(sfa)[ur])
-    bh = dequant_weights(b, sfb, cols=uc)
+    bh = dequant_weights(b, sfb, cols=uc, sfb_gran_n=sfb_gran_n)
     return np.einsum("ik,ik->i", ah[ri], bh[ci])
 
 
-def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices):
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices, sfb_gran_n=BLOCK):
     """Contiguous M-grouped GEMM.
 
     a uint8 [M_total, K], sfa int32 [M_total, KP], b uint8 [G, N, K],
-    sfb int32 [G, ceil(N/128), KP], m_indices int32 [M_total].
+    sfb int32 [G, ceil(N/gran), KP], m_indices int32 [M_total].
     Returns (D float64 [M_total, N] with NaN on undefined rows, valid bool [M_total]).
     """
     b = np.asarray(b, dtype=np.uint8)
@@ -106,11 +122,12 @@ def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices):
         r = np.nonzero(m_indices == g)[0]
         if r.size == 0:
             continue
-        out[r] = dequant_rows(np.asarray(a)[r], np.asarray(sfa)[r]) @ dequant_weights(b[g], np.asarray(sfb)[g]).T
+        out[r] = (dequant_rows(np.asarray(a)[r], np.asarray(sfa)[r])
+                  @ dequant_weights(b[g], np.asarray(sfb)[g], sfb_gran_n=sfb_gran_n).T)
     return out, valid
 
 
-def m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, cols):
+def m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, cols, sfb_gran_n=BLOCK):
     """Sampled outputs of the contiguous GEMM; rows must have a valid expert."""
     m_indices = np.asarray(m_indices, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
@@ -121,7 +138,8 @@ def m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, co
         raise ValueError("sampled rows must belong to an expert")
     for g in np.unique(g_of):
         sel = np.nonzero(g_of == g)[0]
-        out[sel] = fp8_gemm_nt_sampled(a, sfa, np.asarray(b)[g], np.asarray(sfb)[g], rows[sel], cols[sel])
+        out[sel] = fp8_gemm_nt_sampled(a, sfa, np.asarray(b)[g], np.asarray(sfb)[g], rows[sel], cols[sel],
+                                       sfb_gran_n=sfb_gran_n)
     return out
 
 
@@ -131,11 +149,11 @@ def masked_valid_rows(masked_m, G: int, max_m: int) -> np.ndarray:
     return np.arange(max_m)[None, :] < mm[:G, None]
 
 
-def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m):
+def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, sfb_gran_n=BLOCK):
     """Masked M-grouped GEMM.
 
     a uint8 [G, max_m, K], sfa int32 [G, max_m, KP], b uint8 [G, N, K],
-    sfb int32 [G, ceil(N/128), KP], masked_m int32 [G].
+    sfb int32 [G, ceil(N/gran), KP], masked_m int32 [G].
     Returns (D float64 [G, max_m, N] with NaN on undefined rows, valid bool [G, max_m]).
     """
     a = np.asarray(a, dtype=np.uint8)
@@ -147,11 +165,12 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m):
         m = int(valid[g].sum())
         if m == 0:
             continue
-        out[g, :m] = fp8_gemm_nt(a[g, :m], np.asarray(sfa)[g, :m], np.asarray(b)[g], np.asarray(sfb)[g])
+        out[g, :m] = fp8_gemm_nt(a[g, :m], np.asarray(sfa)[g, :m], np.asarray(b)[g], np.asarray(sfb)[g],
+                                 sfb_gran_n=sfb_gran_n)
     return out, valid
 
 
-def m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, groups, rows, cols):
+def m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, groups, rows, cols, sfb_gran_n=BLOCK):
     """Sampled outputs D[groups[i], rows[i], cols[i]] of the masked GEMM (valid rows only)."""
     groups = np.asarray(groups, dtype=np.int64)
     rows = np.asarray(rows, dtype=np.int64)
@@ -160,23 +179,24 @@ def m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, groups, rows, cols):
     for g in np.unique(groups):
         sel = np.nonzero(groups == g)[0]
         out[sel] = fp8_gemm_nt_sampled(np.asarray(a)[g], np.asarray(sfa)[g], np.asarray(b)[g],
-                                       np.asarray(sfb)[g], rows[sel], cols[sel])
+                                       np.asarray(sfb)[g], rows[sel], cols[sel], sfb_gran_n=sfb_gran_n)
     return out
 
 
-def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb) -> np.ndarray:
+def fp8_gemm_nt_points(a_rows, sfa_rows, b_rows, n_idx, sfb, sfb_gran_n=BLOCK) -> np.ndarray:
     """Outputs one at a time: out[i] = sum_k A^_i[k] * B^[n_idx[i], k].
 
     a_rows / sfa_rows: the A rows of the sampled outputs and their packed scale
     rows; b_rows: row n_idx[i] of B for each output; sfb: the full packed scale
-    matrix of that B ([ceil(N/128), KP]), indexed here by n_idx // 128.
+    matrix of that B ([ceil(N/gran), KP]), indexed here by n_idx // gran.
     """
+    gran = _gran(sfb_gran_n)
     A = dequant_rows(a_rows, sfa_rows)
     b_rows = np.asarray(b_rows, dtype=np.uint8)
     P, K = b_rows.shape
     KB = _kb(K)
     n_idx = np.asarray(n_idx, dtype=np.int64)
-    scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))[n_idx // BLOCK]
+    scale = ue8m0_to_f64(unpack_ue8m0(sfb, KB))[n_idx // gran]
     B = (e4m3_to_f64(b_rows).reshape(P, KB, BLOCK) * scale[:, :, None]).reshape(P, K)
     return np.einsum("ik,ik->i", A, B)
 
@@ -203,7 +223,7 @@ def fp8_gemm(a, sfa, b, sfb, layout: str) -> np.ndarray:
 
 # ---- dense GEMM with an accumulation matrix ------------------------------------
 
-def fp8_gemm_nt_acc(a, sfa, b, sfb, c=None) -> np.ndarray:
+def fp8_gemm_nt_acc(a, sfa, b, sfb, c=None, sfb_gran_n=BLOCK) -> np.ndarray:
     """D = C + A^ . B^^T in float64 ("DeepInside DeepGEMM", §4 Hands-on Geek
     Guide: the standard non-grouped FP8 NT GEMM computes D = C + A @ B.T; the
     example passes C as a bf16 [M, N] tensor and the output dtype).
@@ -211,8 +231,8 @@ def fp8_gemm_nt_acc(a, sfa, b, sfb, c=None) -> np.ndarray:
     c: None (C = 0) or the values of C as a float array [M, N] (decoded from
     D's storage type by the caller). Readings: C has D's storage type (bf16 or
     fp32) and is added to the fp32 accumulation before the final conversion,
-    so the reference is the exact sum C + A^.B^^T."""
-    d = fp8_gemm_nt(a, sfa, b, sfb)
+    so the reference is the exact sum C + A^.B^^T. sfb_gran_n as fp8_gemm_nt."""
+    d = fp8_gemm_nt(a, sfa, b, sfb, sfb_gran_n=sfb_gran_n)
     if c is None:
         return d
     c = np.asarray(c, dtype=np.float64)

@@ -133,8 +133,9 @@ def _pack_bytes(byts):
     return w.astype(np.uint32).view(np.int32)
 
 
-def _exact_gemm(a, ea, b, eb):
-    """Exact rational D = A^ B^^T with explicit block loops (no shared code with the oracle)."""
+def _exact_gemm(a, ea, b, eb, gran=128):
+    """Exact rational D = A^ B^^T with explicit block loops (no shared code with the oracle).
+    Row n of B takes scale row n // gran (128x128 blocks, or one row per row of B)."""
     M, K = a.shape
     N = b.shape[0]
     av = torch_e4m3(a)
@@ -145,7 +146,7 @@ def _exact_gemm(a, ea, b, eb):
             acc = Fraction(0)
             for kb in range(K // 128):
                 sa = Fraction(2) ** (int(ea[m, kb]) - 127)
-                sb = Fraction(2) ** (int(eb[n // 128, kb]) - 127)
+                sb = Fraction(2) ** (int(eb[n // gran, kb]) - 127)
                 part = Fraction(0)
                 for kk in range(128):
                     k = kb * 128 + kk
@@ -184,11 +185,11 @@ def test_dense_multi_block_n_exact():
             assert Fraction(got[m, n]) == exact[m][n], (m, n)
 
 
-def one_hot_check(gemm_fn) -> bool:
-    """D of one-hot A rows must be exactly 2^pa * b[n, k_m] * 2^pb(n // 128, k_m // 128)."""
+def one_hot_check(gemm_fn, gran=128) -> bool:
+    """D of one-hot A rows must be exactly 2^pa * b[n, k_m] * 2^pb(n // gran, k_m // 128)."""
     rng = np.random.default_rng(11)
     M, N, K = 6, 300, 640  # 5 K-blocks (ragged packing), 3 N-blocks
-    KB, NB = K // 128, 3
+    KB, NB = K // 128, -(-N // gran)
     ks = np.array([0, 127, 128, 300, 511, 639])
     a = np.zeros((M, K), dtype=np.uint8)
     a[np.arange(M), ks] = 0x38  # 1.0
@@ -201,7 +202,7 @@ def one_hot_check(gemm_fn) -> bool:
     bv = torch_e4m3(b)
     n = np.arange(N)
     for m in range(M):
-        want = (2.0 ** pa[m]) * bv[n, ks[m]] * np.ldexp(1.0, eb[n // 128, ks[m] // 128].astype(np.int64) - 127)
+        want = (2.0 ** pa[m]) * bv[n, ks[m]] * np.ldexp(1.0, eb[n // gran, ks[m] // 128].astype(np.int64) - 127)
         if got.shape != (M, N) or not np.array_equal(got[m], want):
             return False
     return True
@@ -622,5 +623,116 @@ def test_layout_pin_catches_an_unswapped_operand():
     M, K = 128, 128
     a = _rand_codes(rng, (M, K))
     ones = _pack_bytes(np.full((M, 1), 127, np.uint8))
+    ones_b = _pack_bytes(np.full((1, 1), 127, np.uint8))  # one 128x128 block of B
     # reading a [K, M] A as if it were [M, K] changes the result
-    assert not np.array_equal(oracle.fp8_gemm(a, ones, a, ones, "tt"), oracle.fp8_gemm(a, ones, a, ones, "nt"))
+    assert not np.array_equal(oracle.fp8_gemm(a, ones, a, ones_b, "tt"), oracle.fp8_gemm(a, ones, a, ones_b, "nt"))
+
+
+# ------------------------------------ weights with one scale row per row ----
+# "DeepInside DeepGEMM", section 4: the minimal FP8 GEMM example gives B a scale
+# tensor of shape [n, k // 128], one scale per 1x128 block of each row of B.
+
+def _gemm_rows(a, sfa, b, sfb):
+    return oracle.fp8_gemm_nt(a, sfa, b, sfb, sfb_gran_n=1)
+
+
+@pytest.mark.parametrize("M,N,K,seed", [(3, 5, 128, 21), (8, 7, 256, 22), (2, 3, 384, 23)])
+def test_per_row_weight_scales_equal_exact_rational_brute_force(M, N, K, seed):
+    rng = np.random.default_rng(seed)
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    ea = rng.integers(124, 131, size=(M, K // 128)).astype(np.uint8)
+    eb = rng.integers(120, 136, size=(N, K // 128)).astype(np.uint8)
+    got = _gemm_rows(a, _pack_bytes(ea), b, _pack_bytes(eb))
+    exact = _exact_gemm(a, ea, b, eb, gran=1)
+    for m in range(M):
+        for n in range(N):
+            assert Fraction(got[m, n]) == exact[m][n], (m, n)
+
+
+def test_per_row_one_hot_rows_exact():
+    assert one_hot_check(_gemm_rows, gran=1)
+
+
+def test_per_row_scales_repeated_over_blocks_equal_block_scales():
+    # scale rows that repeat each 128x128 block row reduce to the block form
+    rng = np.random.default_rng(24)
+    M, N, K = 5, 300, 512
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(rng.integers(122, 133, size=(M, K // 128)).astype(np.uint8))
+    eb = rng.integers(120, 136, size=(3, K // 128)).astype(np.uint8)
+    block = oracle.fp8_gemm_nt(a, sfa, b, _pack_bytes(eb))
+    rows = _gemm_rows(a, sfa, b, _pack_bytes(np.repeat(eb, 128, axis=0)[:N]))
+    assert np.array_equal(block, rows)
+
+
+def test_per_row_scale_moves_only_its_own_column():
+    # raising the scale bytes of row n0 of B by 3 multiplies column n0 of D by 8
+    # exactly (powers of two) and leaves every other column, including the
+    # rest of n0's 128-row block, unchanged
+    rng = np.random.default_rng(25)
+    M, N, K, n0 = 4, 260, 384, 131
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (N, K))
+    sfa = _pack_bytes(rng.integers(122, 133, size=(M, K // 128)).astype(np.uint8))
+    eb = rng.integers(120, 130, size=(N, K // 128)).astype(np.uint8)
+    d0 = _gemm_rows(a, sfa, b, _pack_bytes(eb))
+    eb2 = eb.copy()
+    eb2[n0] += 3
+    d1 = _gemm_rows(a, sfa, b, _pack_bytes(eb2))
+    others = np.arange(N) != n0
+    assert np.array_equal(d1[:, others], d0[:, others])
+    assert np.array_equal(d1[:, n0], 8.0 * d0[:, n0])
+
+
+def test_per_row_grouped_forms_follow_the_dense_one():
+    rng = np.random.default_rng(26)
+    G, max_m, N, K = 3, 20, 140, 256
+    a = _rand_codes(rng, (G, max_m, K))
+    b = _rand_codes(rng, (G, N, K))
+    sfa = _pack_bytes(rng.integers(122, 133, size=(G * max_m, K // 128)).astype(np.uint8)).reshape(G, max_m, -1)
+    eb = rng.integers(120, 136, size=(G, N, K // 128)).astype(np.uint8)
+    sfb = _pack_bytes(eb.reshape(G * N, -1)).reshape(G, N, -1)
+    mm = np.array([7, 0, 20], dtype=np.int32)
+    d, valid = oracle.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, mm, sfb_gran_n=1)
+    for g in range(G):
+        m = int(mm[g])
+        assert np.array_equal(d[g, :m], _gemm_rows(a[g, :m], sfa[g, :m], b[g], sfb[g]))
+        assert np.all(np.isnan(d[g, m:])) and valid[g].sum() == m
+    # contiguous: the same rows laid end to end, padding rows marked -1
+    idx = np.concatenate([np.full(7, 0), np.full(3, -1), np.full(20, 2)]).astype(np.int32)
+    ac = np.concatenate([a[0, :7], a[1, :3], a[2]])
+    sc = np.concatenate([sfa[0, :7], sfa[1, :3], sfa[2]])
+    dc, vc = oracle.m_grouped_fp8_gemm_nt_contiguous(ac, sc, b, sfb, idx, sfb_gran_n=1)
+    assert np.array_equal(dc[:7], d[0, :7]) and np.array_equal(dc[10:], d[2, :20]) and not vc[7:10].any()
+    pts = oracle.m_grouped_fp8_gemm_nt_masked_sampled(a, sfa, b, sfb, [0, 2, 2], [6, 0, 19], [0, 139, 77],
+                                                      sfb_gran_n=1)
+    assert np.array_equal(pts, [d[0, 6, 0], d[2, 0, 139], d[2, 19, 77]])
+
+
+def test_per_row_granularity_is_checked():
+    a = np.zeros((1, 128), np.uint8)
+    b = np.zeros((130, 128), np.uint8)
+    with pytest.raises(ValueError):
+        oracle.fp8_gemm_nt(a, np.zeros((1, 1), np.int32), b, np.zeros((130, 1), np.int32), sfb_gran_n=64)
+    with pytest.raises(ValueError):  # 2 scale rows cover 130 rows only at granularity 128
+        oracle.fp8_gemm_nt(a, np.zeros((1, 1), np.int32), b, np.zeros((2, 1), np.int32), sfb_gran_n=1)
+
+
+def _planted_rows(kind):
+    """A copy of the per-row oracle with one plausible mistake planted (CPU only)."""
+    def fn(a, sfa, b, sfb):
+        N, K = b.shape
+        KB = K // 128
+        s = oracle.ue8m0_to_f64(oracle.unpack_ue8m0(sfb, KB))
+        n = np.arange(N)
+        idx = {"block_index": n // 128, "next_row": np.minimum(n + 1, N - 1), "first_row": n * 0}[kind]
+        B = (oracle.e4m3_to_f64(b).reshape(N, KB, 128) * s[idx][:, :, None]).reshape(N, K)
+        return og.dequant_rows(a, sfa) @ B.T
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["block_index", "next_row", "first_row"])
+def test_per_row_pins_catch_planted_mistakes(kind):
+    assert not one_hot_check(_planted_rows(kind), gran=1), kind
