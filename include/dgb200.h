@@ -271,6 +271,36 @@ DG_API dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa,
                                        int G, int max_m, int N, int K, void* stream);
 
 /*
+ * The three FP8 forms with a choice of B-scale granularity ("DeepInside
+ * DeepGEMM", section 4: the minimal FP8 GEMM example gives the right-hand
+ * operand one scale row per row, b_sf of shape [n, k / 128]).
+ *   sfb_gran_n : rows of B that share one packed scale row:
+ *                128 -> 128x128 blocks, sfb as in the calls above
+ *                       ([ceil(N/128), KP] per weight matrix);
+ *                1   -> 1x128 blocks, sfb int32 [N, KP] per weight matrix
+ *                       ([G, N, KP] for the grouped forms), row n of B scaled
+ *                       by byte (k / 128) % 4 of word (k / 128) / 4 of row n.
+ *                Any other value returns DG_ERR_INVALID_ARG without launching.
+ * Every other argument, limit, error and property (capture safety, untouched
+ * rows, split-K for the dense form) is that of fp8_gemm_nt_acc,
+ * m_grouped_fp8_gemm_nt_contiguous and m_grouped_fp8_gemm_nt_masked; with
+ * sfb_gran_n = 128 the results are identical to theirs. The scale rows are
+ * read by the scale-producer warp only, so the tile schedule and the main
+ * loop are unchanged.
+ */
+DG_API dg_status fp8_gemm_nt_sfb_gran(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                      int sfb_gran_n, const void* c, void* d, int M, int N, int K, int out_f32,
+                                      void* stream);
+DG_API dg_status m_grouped_fp8_gemm_nt_contiguous_sfb_gran(const void* a, const int32_t* sfa, const void* b,
+                                                           const int32_t* sfb, int sfb_gran_n, void* d,
+                                                           const int32_t* m_indices, int M_total, int N, int K, int G,
+                                                           void* stream);
+DG_API dg_status m_grouped_fp8_gemm_nt_masked_sfb_gran(const void* a, const int32_t* sfa, const void* b,
+                                                       const int32_t* sfb, int sfb_gran_n, void* d,
+                                                       const int32_t* masked_m, int G, int max_m, int N, int K,
+                                                       void* stream);
+
+/*
  * Masked M-grouped BF16 GEMM ("DeepGEMM CUDA Graph Compatibility for Masked
  * Grouped GEMMs", Core Components: the BF16 masked grouped GEMM kernel, and
  * Tensor-Based Metadata Arguments). Plain bf16 operands, no scales; fp32

@@ -26,6 +26,7 @@ __all__ = [
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
     "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc", "quantize_fp8_1x128",
     "fp8_gemm_nn", "fp8_gemm_tn", "fp8_gemm_tt",
+    "fp8_gemm_nt_sfb_gran", "m_grouped_fp8_gemm_nt_contiguous_sfb_gran", "m_grouped_fp8_gemm_nt_masked_sfb_gran",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -101,6 +102,12 @@ def load():
         L.m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_masked.restype = i32
         L.m_grouped_fp8_gemm_nt_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.fp8_gemm_nt_sfb_gran.restype = i32
+        L.fp8_gemm_nt_sfb_gran.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]
+        L.m_grouped_fp8_gemm_nt_contiguous_sfb_gran.restype = i32
+        L.m_grouped_fp8_gemm_nt_contiguous_sfb_gran.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]
+        L.m_grouped_fp8_gemm_nt_masked_sfb_gran.restype = i32
+        L.m_grouped_fp8_gemm_nt_masked_sfb_gran.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]
         L.pack_ue8m0.restype = i32
         L.pack_ue8m0.argtypes = [vp, vp, i64, i32, vp]
         L.pack_ue8m0_validate.restype = i32
@@ -300,6 +307,68 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, max_m=None):
     _check("m_grouped_fp8_gemm_nt_masked",
            load().m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m),
                                                G, max_m, N, K, _stream()))
+    return d
+
+
+def _sfb_rows(N: int, sfb_gran_n: int) -> int:
+    if sfb_gran_n not in (1, BLOCK):
+        raise ValueError(f"sfb_gran_n={sfb_gran_n}: B scale rows cover 1 or {BLOCK} rows of B")
+    return N if sfb_gran_n == 1 else (N + BLOCK - 1) // BLOCK
+
+
+def fp8_gemm_nt_sfb_gran(a, sfa, b, sfb, d, sfb_gran_n: int, c=None):
+    """fp8_gemm_nt_acc with the B-scale granularity given: sfb [N, KP] (sfb_gran_n=1,
+    one scale row per row of b) or [ceil(N/128), KP] (sfb_gran_n=128)."""
+    _need(a, "a", _FP8)
+    M, K = a.shape
+    _need(b, "b", _FP8)
+    N = b.shape[0]
+    _need(b, "b", _FP8, (N, K))
+    _need(sfa, "sfa", _I32, (M, _kp(K)))
+    _need(sfb, "sfb", _I32, (_sfb_rows(N, sfb_gran_n), _kp(K)))
+    _need(d, "d", (torch.bfloat16, torch.float32), (M, N))
+    if c is not None:
+        _need(c, "c", (d.dtype,), (M, N))
+    _check("fp8_gemm_nt_sfb_gran",
+           load().fp8_gemm_nt_sfb_gran(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), int(sfb_gran_n),
+                                       None if c is None else _ptr(c), _ptr(d), M, N, K,
+                                       1 if d.dtype == torch.float32 else 0, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_contiguous_sfb_gran(a, sfa, b, sfb, d, m_indices, sfb_gran_n: int):
+    """m_grouped_fp8_gemm_nt_contiguous with sfb [G, N, KP] (sfb_gran_n=1) or
+    [G, ceil(N/128), KP] (sfb_gran_n=128)."""
+    _need(a, "a", _FP8)
+    M_total, K = a.shape
+    _need(b, "b", _FP8)
+    G, N = b.shape[0], b.shape[1]
+    _need(b, "b", _FP8, (G, N, K))
+    _need(sfa, "sfa", _I32, (M_total, _kp(K)))
+    _need(sfb, "sfb", _I32, (G, _sfb_rows(N, sfb_gran_n), _kp(K)))
+    _need(d, "d", _BF16, (M_total, N))
+    _need(m_indices, "m_indices", _I32, (M_total,))
+    _check("m_grouped_fp8_gemm_nt_contiguous_sfb_gran",
+           load().m_grouped_fp8_gemm_nt_contiguous_sfb_gran(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), int(sfb_gran_n),
+                                                            _ptr(d), _ptr(m_indices), M_total, N, K, G, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_masked_sfb_gran(a, sfa, b, sfb, d, masked_m, sfb_gran_n: int):
+    """m_grouped_fp8_gemm_nt_masked with sfb [G, N, KP] (sfb_gran_n=1) or
+    [G, ceil(N/128), KP] (sfb_gran_n=128)."""
+    _need(a, "a", _FP8)
+    G, max_m, K = a.shape
+    _need(b, "b", _FP8)
+    N = b.shape[1]
+    _need(b, "b", _FP8, (G, N, K))
+    _need(sfa, "sfa", _I32, (G, max_m, _kp(K)))
+    _need(sfb, "sfb", _I32, (G, _sfb_rows(N, sfb_gran_n), _kp(K)))
+    _need(d, "d", _BF16, (G, max_m, N))
+    _need(masked_m, "masked_m", _I32, (G,))
+    _check("m_grouped_fp8_gemm_nt_masked_sfb_gran",
+           load().m_grouped_fp8_gemm_nt_masked_sfb_gran(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), int(sfb_gran_n),
+                                                        _ptr(d), _ptr(masked_m), G, max_m, N, K, _stream()))
     return d
 
 

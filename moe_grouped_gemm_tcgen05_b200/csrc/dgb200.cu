@@ -471,7 +471,7 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.status = st->status;
     p.kb = p.k / (e->dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K per operand row
     p.kp = (p.kb + 3) / 4;
-    p.nb_sf = (p.n + 127) / 128;
+    p.nb_sf = p.sfb_per_row ? p.n : (p.n + 127) / 128;
     p.num_n_blocks = (p.n + bn - 1) / bn;
     if (cg == 2) p.num_m_blocks = (p.rows + 2 * dg::BM - 1) / (2 * dg::BM);
     p.raster_group = 16 / cg;
@@ -536,6 +536,99 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
         choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt, layout, epi);
     return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
                             a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
+}
+
+// Scale rows of B: one per 128x128 block (sfb_gran_n = 128) or one per row of B
+// (sfb_gran_n = 1).
+dg_status sfb_granularity(int sfb_gran_n, int* per_row) {
+    if (sfb_gran_n != 128 && sfb_gran_n != 1) return DG_ERR_INVALID_ARG;
+    *per_row = sfb_gran_n == 1;
+    return DG_OK;
+}
+
+// Dense NT GEMM, D = C + A.B^T. Without C and with a bf16 D it runs the plain
+// epilogue; otherwise the instantiations that add C and/or store fp32.
+dg_status dense_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, int sfb_per_row, const void* c,
+                   void* d, int M, int N, int K, int out_f32, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M <= 0 || (out_f32 != 0 && out_f32 != 1)) return DG_ERR_INVALID_ARG;
+    if (c != nullptr && !aligned(c, 16)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.sfb_per_row = sfb_per_row;
+    p.d = static_cast<__nv_bfloat16*>(d);  // bf16 output (the D tensor map covers it either way)
+    p.d32 = out_f32 ? static_cast<float*>(d) : nullptr;
+    p.out_f32 = out_f32;
+    p.c = c;
+    p.meta = nullptr;
+    p.rows = M;
+    p.n = N;
+    p.k = K;
+    p.groups = 1;
+    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
+    const long long esz = out_f32 ? 4 : 2;
+    const long long bytes = (static_cast<long long>(M) + N) * K + esz * M * N * (c != nullptr ? 2 : 1);
+    const int epi = (c != nullptr || out_f32) ? 1 : 0;
+    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
+                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1, dg::kE4M3, 0, epi);
+}
+
+dg_status contiguous_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, int sfb_per_row,
+                        void* d, const int32_t* m_indices, int M_total, int N, int K, int G, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M_total <= 0 || G <= 0 || m_indices == nullptr) return DG_ERR_INVALID_ARG;
+    if (!aligned(m_indices, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.sfb_per_row = sfb_per_row;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = m_indices;
+    p.rows = M_total;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (M_total + dg::BM - 1) / dg::BM;
+    const long long bytes = static_cast<long long>(M_total) * K + static_cast<long long>(G) * N * K +
+                            2LL * M_total * N;
+    return launch_gemm(dg::kContiguous, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 3,
+                       static_cast<uint64_t>(M_total), 1, static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+}
+
+dg_status masked_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, int sfb_per_row, void* d,
+                    const int32_t* masked_m, int G, int max_m, int N, int K, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (G <= 0 || max_m <= 0 || masked_m == nullptr) return DG_ERR_INVALID_ARG;
+    if (G > dg::MAX_MASKED_GROUPS) return DG_ERR_UNSUPPORTED;
+    if (!aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.sfb_per_row = sfb_per_row;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = masked_m;
+    p.rows = max_m;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (max_m + dg::BM - 1) / dg::BM;
+    const long long mb_total = static_cast<long long>(G) * p.num_m_blocks;
+    const long long bytes = static_cast<long long>(G) * N * K;  // the weights; the valid rows are unknown here
+    return launch_gemm(dg::kMasked, p, mb_total, mb_total, bytes, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
+                       static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
 }
 
 }  // namespace
@@ -609,25 +702,7 @@ dg_status dgb200_set_test_hooks(int mode, int wait_limit_ms) {
 
 dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M, int N,
                       int K, void* stream) {
-    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
-    if (s != DG_OK) return s;
-    if (M <= 0) return DG_ERR_INVALID_ARG;
-    DeviceState* st = nullptr;
-    if ((s = current_device(&st)) != DG_OK) return s;
-    GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.sfa = sfa;
-    p.sfb = sfb;
-    p.d = static_cast<__nv_bfloat16*>(d);
-    p.meta = nullptr;
-    p.rows = M;
-    p.n = N;
-    p.k = K;
-    p.groups = 1;
-    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
-    const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
-    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
-                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1);
+    return dense_nt(a, sfa, b, sfb, 0, nullptr, d, M, N, K, 0, stream);
 }
 
 // Dense GEMM in the TN/NN/TT layouts (layout bit 0: A stored [K, M]; bit 1: B
@@ -672,30 +747,15 @@ dg_status fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const in
 
 dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const void* c, void* d,
                           int M, int N, int K, int out_f32, void* stream) {
-    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    return dense_nt(a, sfa, b, sfb, 0, c, d, M, N, K, out_f32, stream);
+}
+
+dg_status fp8_gemm_nt_sfb_gran(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, int sfb_gran_n,
+                               const void* c, void* d, int M, int N, int K, int out_f32, void* stream) {
+    int per_row = 0;
+    const dg_status s = sfb_granularity(sfb_gran_n, &per_row);
     if (s != DG_OK) return s;
-    if (M <= 0 || (out_f32 != 0 && out_f32 != 1)) return DG_ERR_INVALID_ARG;
-    if (c != nullptr && !aligned(c, 16)) return DG_ERR_ALIGNMENT;
-    DeviceState* st = nullptr;
-    if ((s = current_device(&st)) != DG_OK) return s;
-    GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.sfa = sfa;
-    p.sfb = sfb;
-    p.d = static_cast<__nv_bfloat16*>(d);  // bf16 output (the D tensor map covers it either way)
-    p.d32 = out_f32 ? static_cast<float*>(d) : nullptr;
-    p.out_f32 = out_f32;
-    p.c = c;
-    p.meta = nullptr;
-    p.rows = M;
-    p.n = N;
-    p.k = K;
-    p.groups = 1;
-    p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
-    const long long esz = out_f32 ? 4 : 2;
-    const long long bytes = (static_cast<long long>(M) + N) * K + esz * M * N * (c != nullptr ? 2 : 1);
-    return launch_gemm(dg::kDense, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 2,
-                       static_cast<uint64_t>(M), 1, static_cast<uint64_t>(N), 1, dg::kE4M3, 0, 1);
+    return dense_nt(a, sfa, b, sfb, per_row, c, d, M, N, K, out_f32, stream);
 }
 
 dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
@@ -751,53 +811,31 @@ dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, 
 dg_status m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
                                            void* d, const int32_t* m_indices, int M_total, int N, int K, int G,
                                            void* stream) {
-    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    return contiguous_nt(a, sfa, b, sfb, 0, d, m_indices, M_total, N, K, G, stream);
+}
+
+dg_status m_grouped_fp8_gemm_nt_contiguous_sfb_gran(const void* a, const int32_t* sfa, const void* b,
+                                                    const int32_t* sfb, int sfb_gran_n, void* d,
+                                                    const int32_t* m_indices, int M_total, int N, int K, int G,
+                                                    void* stream) {
+    int per_row = 0;
+    const dg_status s = sfb_granularity(sfb_gran_n, &per_row);
     if (s != DG_OK) return s;
-    if (M_total <= 0 || G <= 0 || m_indices == nullptr) return DG_ERR_INVALID_ARG;
-    if (!aligned(m_indices, 4)) return DG_ERR_ALIGNMENT;
-    DeviceState* st = nullptr;
-    if ((s = current_device(&st)) != DG_OK) return s;
-    GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.sfa = sfa;
-    p.sfb = sfb;
-    p.d = static_cast<__nv_bfloat16*>(d);
-    p.meta = m_indices;
-    p.rows = M_total;
-    p.n = N;
-    p.k = K;
-    p.groups = G;
-    p.num_m_blocks = (M_total + dg::BM - 1) / dg::BM;
-    const long long bytes = static_cast<long long>(M_total) * K + static_cast<long long>(G) * N * K +
-                            2LL * M_total * N;
-    return launch_gemm(dg::kContiguous, p, p.num_m_blocks, p.num_m_blocks, bytes, stream, st, a, b, 2, 3,
-                       static_cast<uint64_t>(M_total), 1, static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+    return contiguous_nt(a, sfa, b, sfb, per_row, d, m_indices, M_total, N, K, G, stream);
 }
 
 dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
                                        const int32_t* masked_m, int G, int max_m, int N, int K, void* stream) {
-    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    return masked_nt(a, sfa, b, sfb, 0, d, masked_m, G, max_m, N, K, stream);
+}
+
+dg_status m_grouped_fp8_gemm_nt_masked_sfb_gran(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                                int sfb_gran_n, void* d, const int32_t* masked_m, int G, int max_m,
+                                                int N, int K, void* stream) {
+    int per_row = 0;
+    const dg_status s = sfb_granularity(sfb_gran_n, &per_row);
     if (s != DG_OK) return s;
-    if (G <= 0 || max_m <= 0 || masked_m == nullptr) return DG_ERR_INVALID_ARG;
-    if (G > dg::MAX_MASKED_GROUPS) return DG_ERR_UNSUPPORTED;
-    if (!aligned(masked_m, 4)) return DG_ERR_ALIGNMENT;
-    DeviceState* st = nullptr;
-    if ((s = current_device(&st)) != DG_OK) return s;
-    GemmParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.sfa = sfa;
-    p.sfb = sfb;
-    p.d = static_cast<__nv_bfloat16*>(d);
-    p.meta = masked_m;
-    p.rows = max_m;
-    p.n = N;
-    p.k = K;
-    p.groups = G;
-    p.num_m_blocks = (max_m + dg::BM - 1) / dg::BM;
-    const long long mb_total = static_cast<long long>(G) * p.num_m_blocks;
-    const long long bytes = static_cast<long long>(G) * N * K;  // the weights; the valid rows are unknown here
-    return launch_gemm(dg::kMasked, p, mb_total, mb_total, bytes, stream, st, a, b, 3, 3, static_cast<uint64_t>(max_m),
-                       static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+    return masked_nt(a, sfa, b, sfb, per_row, d, masked_m, G, max_m, N, K, stream);
 }
 
 dg_status m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d, const int32_t* masked_m, int G,

@@ -89,7 +89,7 @@ struct GemmParams {
     CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped); box BN/CG rows
     CUtensorMap tma_d;        // D (bf16, store): 2-D {N, rows} or 3-D {N, max_m, G}; 32x32 box, 64-byte swizzle
     const int32_t* sfa;       // packed scale rows of A
-    const int32_t* sfb;       // packed scale rows of B (per 128 rows, per group)
+    const int32_t* sfb;       // packed scale rows of B (per 128 rows or per row, per group)
     __nv_bfloat16* d;         // output
     const int32_t* meta;      // m_indices (contiguous) / masked_m (masked) / null
     uint32_t* status;         // device status word
@@ -97,7 +97,8 @@ struct GemmParams {
     int n, k, groups;
     int kb;                   // K / 128
     int kp;                   // ceil(kb / 4) packed words per scale row
-    int nb_sf;                // ceil(N / 128) scale rows per weight matrix
+    int nb_sf;                // scale rows per weight matrix: ceil(N / 128), or N when sfb_per_row
+    int sfb_per_row;          // 1: one scale row per row of B (1x128 blocks); 0: per 128x128 block
     int num_m_blocks;         // ceil(rows / (128 * CG)) m-tiles
     int num_n_blocks;         // ceil(N / BN)
     int raster_group;         // m-tiles per raster band (dense / contiguous)
@@ -336,7 +337,8 @@ __device__ __forceinline__ int rot_group(const GemmParams& p, int t, int gi, int
 
 // Scale words of one 4-K-block group of a tile: lane r holds, for j = 0..3,
 // the word of A row row0 + 32j + r and, per 128-column chunk, the word of B
-// column n0 + 128*chunk + 32j + r. Stored as one 16-byte row per lane, this is
+// column n0 + 128*chunk + 32j + r (from the scale row of its 128x128 block, or
+// its own scale row when B is scaled per row). Stored as one 16-byte row per lane, this is
 // the 32x128-bit matrix whose copy to TMEM puts row m at lane m % 32, column
 // m / 32. For a CTA pair (CG = 2) the words of the second CTA's 128 rows are
 // gathered too (`ap`), by the leader, which stores them into the peer's slot.
@@ -367,7 +369,7 @@ struct ScaleWords {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int col = n0 + 128 * ch + 32 * j + static_cast<int>(lane);
-                const int nb = min(col / 128, p.nb_sf - 1);
+                const int nb = min(p.sfb_per_row ? col : col / 128, p.nb_sf - 1);
                 b[ch][j] = static_cast<uint32_t>(__ldg(sfb + static_cast<size_t>(nb) * p.kp + kg));
             }
         }

@@ -13,6 +13,11 @@ s = 2^ceil(log2(max(amax, 1e-4) / 448)) and the stored byte is
 saturates). Scales are returned as fp32 powers of two, i.e. valid UE8M0
 inputs to the pack step.
 
+Weights scaled per row (``sfb_gran_n=1``: one scale per 1x128 block of each row
+of B, scales [N, K/128]) are quantised like activations; before quantisation
+each row of B is multiplied by 2^u, u uniform on {-3..3}, so that neighbouring
+scale rows differ as per-channel weight scales do.
+
 Workloads (seed = 1000 + workload number, numpy PCG64):
   0  dense M=128, N=256, K=512
   1  dense M in {64, 4096} x (N, K) in {(2112,7168), (24576,1536), (7168,16384), (4096,7168)}
@@ -81,24 +86,37 @@ def _normal(rng, shape):
     return rng.standard_normal(size=shape, dtype=np.float32)
 
 
-def dense(M: int, N: int, K: int, seed: int):
-    """Dense NT problem: a [M,K], sfa_f32 [M,K/128], b [N,K], sfb_f32 [ceil(N/128),K/128]."""
+def quantise_weights(rng, N: int, K: int, sfb_gran_n: int = BLOCK):
+    """Random weights [N, K] quantised per 128x128 block (sfb_gran_n=128) or per
+    1x128 block of each row (sfb_gran_n=1, with the per-row spread above)."""
+    w = _normal(rng, (N, K))
+    if sfb_gran_n == BLOCK:
+        return quantise_blocks(w)
+    if sfb_gran_n != 1:
+        raise ValueError(f"sfb_gran_n={sfb_gran_n}")
+    spread = np.ldexp(1.0, rng.integers(-3, 4, size=N)).astype(np.float32)
+    return quantise_rows(w * spread[:, None])
+
+
+def dense(M: int, N: int, K: int, seed: int, sfb_gran_n: int = BLOCK):
+    """Dense NT problem: a [M,K], sfa_f32 [M,K/128], b [N,K], sfb_f32 [ceil(N/gran),K/128]."""
     rng = rng_for(seed)
     a, sfa = quantise_rows(_normal(rng, (M, K)))
-    b, sfb = quantise_blocks(_normal(rng, (N, K)))
+    b, sfb = quantise_weights(rng, N, K, sfb_gran_n)
     return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, M=M, N=N, K=K)
 
 
-def grouped_weights(rng, G: int, N: int, K: int):
+def grouped_weights(rng, G: int, N: int, K: int, sfb_gran_n: int = BLOCK):
     bs, sfbs = [], []
     for _ in range(G):
-        b, sfb = quantise_blocks(_normal(rng, (N, K)))
+        b, sfb = quantise_weights(rng, N, K, sfb_gran_n)
         bs.append(b)
         sfbs.append(sfb)
     return np.stack(bs), np.stack(sfbs)
 
 
-def contiguous(counts, N: int, K: int, seed: int, align: int = BLOCK, tail_blocks: int = 0):
+def contiguous(counts, N: int, K: int, seed: int, align: int = BLOCK, tail_blocks: int = 0,
+               sfb_gran_n: int = BLOCK):
     """Contiguous M-grouped problem.
 
     Expert g owns ``counts[g]`` real rows, padded with -1 rows up to a multiple
@@ -120,12 +138,13 @@ def contiguous(counts, N: int, K: int, seed: int, align: int = BLOCK, tail_block
     qa, qs = quantise_rows(_normal(rng, (int(valid.sum()), K)))
     a[valid] = qa
     sfa[valid] = qs
-    b, sfb = grouped_weights(rng, G, N, K)
+    b, sfb = grouped_weights(rng, G, N, K, sfb_gran_n)
     return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, m_indices=m_indices,
                 M_total=M_total, N=N, K=K, G=G)
 
 
-def masked(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bool = True):
+def masked(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bool = True,
+           sfb_gran_n: int = BLOCK):
     """Masked M-grouped problem: a [G,max_m,K], b [G,N,K]; rows >= masked_m hold NaN bytes."""
     rng = rng_for(seed)
     masked_m = np.asarray(masked_m, dtype=np.int32)
@@ -137,7 +156,7 @@ def masked(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bo
     if fill_invalid_nan:
         rows = np.arange(max_m)[None, :] >= np.clip(masked_m, 0, max_m)[:, None]
         a[rows] = NAN_BYTE
-    b, sfb = grouped_weights(rng, G, N, K)
+    b, sfb = grouped_weights(rng, G, N, K, sfb_gran_n)
     return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, masked_m=masked_m,
                 G=G, max_m=max_m, N=N, K=K)
 

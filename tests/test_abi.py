@@ -68,6 +68,33 @@ def test_host_argument_checks_fail_before_device_work(lib):
     assert p(vp(0x10002), good, 4, 4, None) == 2
 
 
+def test_sfb_granularity_is_checked_on_the_host(lib):
+    vp, i = ctypes.c_void_p, ctypes.c_int
+    good = vp(0x10000)
+    f = lib.fp8_gemm_nt_sfb_gran
+    f.restype = i
+    f.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, i, vp]
+    for gran in (0, 2, 64, 127, 256, -1):
+        assert f(good, good, good, good, gran, None, good, 128, 128, 128, 0, None) == 1, gran
+    assert f(good, good, good, good, 1, None, good, 128, 128, 100, 0, None) == 1      # K % 128
+    assert f(good, good, good, good, 1, None, good, 128, 128, 128, 2, None) == 1      # out_f32 not 0 / 1
+    c = lib.m_grouped_fp8_gemm_nt_contiguous_sfb_gran
+    c.restype = i
+    c.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, i, vp]
+    assert c(good, good, good, good, 64, good, good, 128, 128, 128, 2, None) == 1
+    assert c(good, good, good, good, 1, good, None, 128, 128, 128, 2, None) == 1      # null m_indices
+    m = lib.m_grouped_fp8_gemm_nt_masked_sfb_gran
+    m.restype = i
+    m.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, i, vp]
+    assert m(good, good, good, good, 3, good, good, 4, 64, 128, 128, None) == 1
+    assert m(good, good, good, good, 1, good, good, 2048, 64, 128, 128, None) == 3    # too many groups
+    import torch
+    x = torch.zeros((128, 128), dtype=torch.uint8)
+    with pytest.raises(ValueError):  # the binding checks the scale-row count for the granularity
+        dg.fp8_gemm_nt_sfb_gran(x, torch.zeros((128, 1), dtype=torch.int32), x,
+                                torch.zeros((1, 1), dtype=torch.int32), torch.zeros((128, 128), dtype=torch.bfloat16), 1)
+
+
 def test_binding_fails_loudly_without_cuda():
     import torch
     if torch.cuda.is_available():
