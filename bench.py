@@ -425,7 +425,20 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
         out[f"dense_{name}_{M}x{N}x{K}"] = {"us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
                                             "roofline_frac": frac_tensor_mem(fl, dense_bytes(M, N, K), ms),
                                             "bound": "tensor"}
-    del p, sfa, sfb, d, a_km, b_kn
+    # the same NT problem with one weight scale row per row of B (sfb [N, KP])
+    sfb_rows = sfb.repeat_interleave(128, dim=0)[:N].contiguous()
+    op = lambda: dg.fp8_gemm_nt_sfb_gran(p["a"], sfa, p["b"], sfb_rows, d, 1)
+    op()
+    g = EventGraph([op] * 4)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(g.durations_ms())
+    g.close()
+    fl = gemm_flops(M, N, K)
+    out[f"dense_sfb_per_row_{M}x{N}x{K}"] = {"us": ms * 1e3, "TFLOP/s": fl / ms / 1e9,
+                                              "roofline_frac": frac_tensor_mem(fl, dense_bytes(M, N, K), ms),
+                                              "bound": "tensor"}
+    del p, sfa, sfb, sfb_rows, d, a_km, b_kn
 
     # per-token FP8 quantiser: bf16 activations [4096, 7168] -> E4M3 + packed UE8M0
     rows, K = 4096, 7168

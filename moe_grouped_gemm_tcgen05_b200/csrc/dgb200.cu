@@ -88,6 +88,16 @@ const int g_k_rotate = [] {
     const char* v = std::getenv("DGB200_K_ROTATE");
     return (v != nullptr && v[0] == '1') ? 1 : 0;
 }();
+// With B scaled per row, scale rows whose length is a multiple of 4 words, on
+// 16-byte aligned bases, are read 16 bytes (four K groups) per row at a time
+// when the K groups are walked in order; DGB200_SF_VEC4=0 reads one word per
+// group instead. Measured on 4096x7168x16384 (BN 224, CTA pairs): per-row B
+// scales 370 -> 335 us; with 128x128 B blocks (one broadcast word per 128
+// columns) the one-word reads are faster, 311 vs 325 us, so they keep them.
+const bool g_sf_vec4 = [] {
+    const char* v = std::getenv("DGB200_SF_VEC4");
+    return !(v != nullptr && v[0] == '0');
+}();
 
 // --------------------------------------------------------------- kernels ----
 
@@ -472,6 +482,11 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.kb = p.k / (e->dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K per operand row
     p.kp = (p.kb + 3) / 4;
     p.nb_sf = p.sfb_per_row ? p.n : (p.n + 127) / 128;
+    // 16-byte reads of the scale rows need every row to start on a 16-byte boundary
+    p.sf_vec4 = (p.sfb_per_row && e->dt == dg::kE4M3 && g_sf_vec4 && p.kp % 4 == 0 && aligned(p.sfa, 16) &&
+                 aligned(p.sfb, 16))
+                    ? 1
+                    : 0;
     p.num_n_blocks = (p.n + bn - 1) / bn;
     if (cg == 2) p.num_m_blocks = (p.rows + 2 * dg::BM - 1) / (2 * dg::BM);
     p.raster_group = 16 / cg;
@@ -481,6 +496,7 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.ws = choice.splits > 1 ? ws : nullptr;
     p.counters = choice.splits > 1 ? counters : nullptr;
     p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
+    if (p.k_rotate) p.sf_vec4 = 0;                     // quads are walked in K order
     if (e->layout & 1) {
         if (!encode_mnmajor(&p.tma_a, a, a_rows, static_cast<uint64_t>(p.k))) return DG_ERR_INVALID_ARG;
     } else if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128, e->dt)) {

@@ -105,6 +105,8 @@ struct GemmParams {
     uint64_t wait_limit_ns;   // bound of every mbarrier wait
     int k_rotate;             // 1: each tile walks its K groups starting at group (tile mod groups)
     int test_mode;            // 1: CTA 0 withholds its first scale-group arrive (exercises the timeout path)
+    int sf_vec4;              // 1: scale rows are read 16 bytes (4 K groups) at a time (B scaled per row,
+                              //    kp % 4 == 0, 16-byte bases, K groups in order)
     // split-K (dense form, single CTAs): each output tile is computed by `splits`
     // work units over disjoint ranges of K groups; the last one to finish adds
     // the fp32 partials in split order and writes the bf16 tile
@@ -391,6 +393,66 @@ struct ScaleWords {
             for (int ch = 0; ch < CH; ++ch)
                 st_cluster_v4(sfb_slot_peer + 512u * ch + 16u * lane, b[ch][0], b[ch][1], b[ch][2], b[ch][3]);
         }
+    }
+};
+
+// Scale words of four consecutive K groups (one 16-byte load per scale row),
+// for packed rows whose length is a multiple of four words on 16-byte
+// aligned bases. Same rows and columns as ScaleWords; `base` is the first of
+// the four groups (a multiple of 4). One such load serves four groups, so the
+// scattered row reads are a quarter of the one-word loads: this pays when B
+// is scaled per row, where every column reads its own scale row.
+template <int BN, int KIND, int CG>
+struct ScaleQuads {
+    static constexpr int CH = (BN + 127) / 128;
+    uint4 a[4];
+    uint4 ap[CG == 2 ? 4 : 1];
+    uint4 b[CH][4];
+    int lo, hi;  // the groups [lo, hi) of the tile that this quad serves
+
+    __device__ __forceinline__ static const uint4* at(const int32_t* row_start, int base) {
+        return reinterpret_cast<const uint4*>(row_start + base);
+    }
+
+    __device__ __forceinline__ void load(const GemmParams& p, int row0, int n0, int g, int base, uint32_t lane) {
+        size_t row_base = 0;
+        if constexpr (KIND == kMasked) row_base = static_cast<size_t>(g) * p.rows;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int r = min(row0 + 32 * j + static_cast<int>(lane), p.rows - 1);
+            a[j] = __ldg(at(p.sfa + (row_base + r) * p.kp, base));
+            if constexpr (CG == 2) {
+                const int rp = min(row0 + BM + 32 * j + static_cast<int>(lane), p.rows - 1);
+                ap[j] = __ldg(at(p.sfa + (row_base + rp) * p.kp, base));
+            }
+        }
+        const int32_t* sfb = p.sfb + static_cast<size_t>(KIND == kDense ? 0 : max(g, 0)) * p.nb_sf * p.kp;
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int col = n0 + 128 * ch + 32 * j + static_cast<int>(lane);
+                const int nb = min(p.sfb_per_row ? col : col / 128, p.nb_sf - 1);
+                b[ch][j] = __ldg(at(sfb + static_cast<size_t>(nb) * p.kp, base));
+            }
+        }
+    }
+
+    __device__ __forceinline__ static uint32_t pick(const uint4& v, int i) {
+        return static_cast<uint32_t>(i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w)));
+    }
+
+    // the words of group base + i
+    __device__ __forceinline__ void words(ScaleWords<BN, KIND, CG>& w, int i) const {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            w.a[j] = pick(a[j], i);
+            if constexpr (CG == 2) w.ap[j] = pick(ap[j], i);
+        }
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w.b[ch][j] = pick(b[ch][j], i);
     }
 };
 
@@ -684,15 +746,54 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 if (++slot == SF_RING) { slot = 0; sf_phase ^= 1u; }
                 return true;
             };
-            ScaleWords<BN, KIND, CG> w0, w1;
-            bool v0 = load_next(w0);
-            bool v1 = load_next(w1);
-            while (v0) {
-                if (!put(w0)) break;
-                v0 = load_next(w0);
-                if (!v1) break;
-                if (!put(w1)) break;
-                v1 = load_next(w1);
+            if (p.sf_vec4) {
+                // 16-byte rows of scale words (K groups in order, no rotation):
+                // quads of four groups are walked tile by tile, each serving
+                // the groups of its tile that it covers; the loads of the next
+                // quad are in flight while the current one is stored
+                int q_base = cok ? (ctile.kg0 & ~3) : 0;
+                auto load_quad = [&](ScaleQuads<BN, KIND, CG>& q) -> bool {
+                    if (!cok) return false;
+                    q.lo = max(q_base, ctile.kg0);
+                    q.hi = min(q_base + 4, ctile.kg1);
+                    q.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, q_base, lane);
+                    q_base += 4;
+                    if (q_base >= ctile.kg1) {
+                        ct += units;
+                        cok = next_tile<KIND, true, CG>(p, s_prefix, s_mm, ct, units, cg_cur, ctile, lane);
+                        if (cok) q_base = ctile.kg0 & ~3;
+                    }
+                    return true;
+                };
+                auto put_quad = [&](const ScaleQuads<BN, KIND, CG>& q) -> bool {
+                    for (int kg = q.lo; kg < q.hi; ++kg) {
+                        ScaleWords<BN, KIND, CG> w;
+                        q.words(w, kg & 3);
+                        if (!put(w)) return false;
+                    }
+                    return true;
+                };
+                ScaleQuads<BN, KIND, CG> q0, q1;
+                bool h0 = load_quad(q0);
+                bool h1 = load_quad(q1);
+                while (h0) {
+                    if (!put_quad(q0)) break;
+                    h0 = load_quad(q0);
+                    if (!h1) break;
+                    if (!put_quad(q1)) break;
+                    h1 = load_quad(q1);
+                }
+            } else {
+                ScaleWords<BN, KIND, CG> w0, w1;
+                bool v0 = load_next(w0);
+                bool v1 = load_next(w1);
+                while (v0) {
+                    if (!put(w0)) break;
+                    v0 = load_next(w0);
+                    if (!v1) break;
+                    if (!put(w1)) break;
+                    v1 = load_next(w1);
+                }
             }
         }
     } else if (warp == 1) {

@@ -172,3 +172,70 @@ def test_contiguous_parity_and_padding(cg):
     sent = is_sentinel(d)
     assert sent[~valid].all(), "padding rows were written"
     check_fp(bf16_to_f64(d)[valid], ref[valid], f"contiguous, per-row B scales, cg={cg}")
+
+
+# ---- 16-byte scale-row reads vs one-word reads ----------------------------------
+# With B scaled per row, packed scale rows of a multiple of four words on 16-byte
+# aligned bases are read four K groups at a time; the same scales at a 4-byte
+# offset take the one-word path. Both must give identical bits (granularity 128
+# compares the one-word path with itself at two alignments).
+
+def _offset_copy(t):
+    """The same values in a buffer that starts 4 bytes past a 16-byte boundary."""
+    buf = torch.empty(t.numel() + 1, dtype=t.dtype, device=t.device)
+    v = buf[1:].view(t.shape)
+    v.copy_(t)
+    assert v.data_ptr() % 16 == 4
+    return v
+
+
+@pytest.mark.parametrize("gran,bn,cg,splits", [(128, 0, 0, 0), (1, 0, 0, 0), (128, 128, 2, 0), (1, 224, 2, 0),
+                                               (128, 64, 1, 5), (1, 96, 1, 5), (1, 256, 1, 3)])
+def test_vector_scale_reads_equal_word_reads_dense(gran, bn, cg, splits):
+    # K = 6144: 12 packed words per row; 5 split ranges start at groups 0, 2, 4, 7, 9
+    M, N, K = 300 if splits == 0 else 64, 392, 6144
+    p = W.dense(M, N, K, seed=200 + bn + splits + gran, sfb_gran_n=gran)
+    a, b = _dev(p["a"]), _dev(p["b"])
+    sfa, sfb = dg.pack_ue8m0(_dev(p["sfa_f32"])), dg.pack_ue8m0(_dev(p["sfb_f32"]))
+    assert sfa.data_ptr() % 16 == 0 and sfb.data_ptr() % 16 == 0 and sfa.shape[1] % 4 == 0
+    dg.set_block_n(bn)
+    dg.set_cta_group(cg)
+    dg.set_splits(splits)
+    d0 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    d1 = torch.empty_like(d0)
+    dg.fp8_gemm_nt_sfb_gran(a, sfa, b, sfb, d0, gran)
+    dg.fp8_gemm_nt_sfb_gran(a, _offset_copy(sfa), b, _offset_copy(sfb), d1, gran)
+    torch.cuda.synchronize()
+    assert torch.equal(d0.view(torch.int16), d1.view(torch.int16))
+    check_fp(bf16_to_f64(d0), _ref(p) if gran == 1 else
+             oracle.fp8_gemm_nt(p["a"], _opack(p["sfa_f32"]), p["b"], _opack(p["sfb_f32"])), "16-byte scale reads")
+
+
+@pytest.mark.parametrize("gran", [128, 1])
+def test_vector_scale_reads_equal_word_reads_grouped(gran):
+    mm = np.array([1, 0, 129, 256, 67], dtype=np.int32)
+    q = W.masked(mm, 256, 264, 2048, seed=210 + gran, sfb_gran_n=gran)
+    args = [_dev(q["a"]), dg.pack_ue8m0(_dev(q["sfa_f32"])), _dev(q["b"]), dg.pack_ue8m0(_dev(q["sfb_f32"]))]
+    m0 = fill_sentinel(torch.empty((5, 256, 264), dtype=torch.bfloat16, device="cuda"))
+    m1 = fill_sentinel(torch.empty_like(m0))
+    mmd = _dev(mm)
+    dg.m_grouped_fp8_gemm_nt_masked_sfb_gran(*args, m0, mmd, gran)
+    dg.m_grouped_fp8_gemm_nt_masked_sfb_gran(args[0], _offset_copy(args[1]), args[2], _offset_copy(args[3]), m1, mmd,
+                                             gran)
+    torch.cuda.synchronize()
+    assert torch.equal(m0.view(torch.int16), m1.view(torch.int16))
+    ref, valid = oracle.m_grouped_fp8_gemm_nt_masked(q["a"], _opack(q["sfa_f32"]), q["b"], _opack(q["sfb_f32"]), mm,
+                                                     sfb_gran_n=gran)
+    check_fp(bf16_to_f64(m0)[valid], ref[valid], "masked, 16-byte scale reads")
+    for cg in (1, 2):
+        c = W.contiguous([130, 0, 300], 264, 4096, seed=220 + gran + cg, sfb_gran_n=gran)
+        args = [_dev(c["a"]), dg.pack_ue8m0(_dev(c["sfa_f32"])), _dev(c["b"]), dg.pack_ue8m0(_dev(c["sfb_f32"]))]
+        dg.set_cta_group(cg)
+        c0 = fill_sentinel(torch.empty((c["M_total"], 264), dtype=torch.bfloat16, device="cuda"))
+        c1 = fill_sentinel(torch.empty_like(c0))
+        idx = _dev(c["m_indices"])
+        dg.m_grouped_fp8_gemm_nt_contiguous_sfb_gran(*args, c0, idx, gran)
+        dg.m_grouped_fp8_gemm_nt_contiguous_sfb_gran(args[0], _offset_copy(args[1]), args[2], _offset_copy(args[3]),
+                                                     c1, idx, gran)
+        torch.cuda.synchronize()
+        assert torch.equal(c0.view(torch.int16), c1.view(torch.int16)), cg
