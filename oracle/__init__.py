@@ -17,7 +17,8 @@ ue8m0  -- UE8M0 scale bytes: decode, the capture-safe pack of fp32 scales
           into four bytes per int32, the matching unpack, and the optional
           eager validator
 gemm   -- dequantise-and-multiply references for the dense NT GEMM and the
-          contiguous / masked M-grouped GEMMs, and the BF16 masked grouped GEMM
+          contiguous / masked / psum_m-driven M-grouped GEMMs, and the BF16
+          masked grouped GEMM
 
 Sources (web pages about DeepGEMM):
   [P1] "DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs:
@@ -51,6 +52,8 @@ from .gemm import (  # noqa: F401
     m_grouped_fp8_gemm_nt_masked,
     m_grouped_fp8_gemm_nt_masked_sampled,
     masked_valid_rows,
+    psum_group_rows,
+    m_grouped_fp8_gemm_nt_psum,
     m_grouped_bf16_gemm_nt_masked,
     m_grouped_bf16_gemm_nt_masked_sampled,
 )

@@ -28,6 +28,9 @@ the call shape):
 * contiguous: rows of A are concatenated by expert; ``m_indices[r]`` gives the
   expert of row r. Rows with an index outside [0, G) (-1 marks padding) are
   not computed and their output is left as it was.
+* psum_m-driven (same page, Tensor-Based Metadata Arguments; reading in
+  psum_group_rows): A is [M_total, K] with the groups' rows end to end, group
+  g owning rows [psum_m[g-1], psum_m[g]); rows in no group are left as they were.
 * masked ("DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs",
   Tensor-Based Metadata Arguments and the FAQ on dynamic shapes): A is
   [G, max_m, K] and D is [G, max_m, N]; only the first masked_m[g] rows of group
@@ -141,6 +144,49 @@ def m_grouped_fp8_gemm_nt_contiguous_sampled(a, sfa, b, sfb, m_indices, rows, co
         out[sel] = fp8_gemm_nt_sampled(a, sfa, np.asarray(b)[g], np.asarray(sfb)[g], rows[sel], cols[sel],
                                        sfb_gran_n=sfb_gran_n)
     return out
+
+
+def psum_group_rows(psum_m, M_total: int):
+    """Row range [start_g, end_g) of every group of the psum_m-driven grouped GEMM.
+
+    Reading ("DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs",
+    Tensor-Based Metadata Arguments, names psum_m as device metadata of the
+    grouped GEMMs without defining it): psum_m[g] is the inclusive prefix sum
+    of the groups' row counts, so group g owns rows [psum_m[g-1], psum_m[g])
+    of an unpadded A [M_total, K] (psum_m[-1] = 0). Malformed values are made
+    harmless: end_g = min(max(0, psum_m[0], ..., psum_m[g]), M_total) and
+    start_g = end_{g-1}, start_0 = 0, so a decreasing entry gives an empty
+    group and no row belongs to two groups.
+    """
+    psum_m = np.asarray(psum_m, dtype=np.int64)
+    ends = np.minimum(np.maximum.accumulate(np.maximum(psum_m, 0)), M_total)
+    starts = np.concatenate([[0], ends[:-1]]).astype(np.int64)
+    return starts, ends
+
+
+def m_grouped_fp8_gemm_nt_psum(a, sfa, b, sfb, psum_m, sfb_gran_n=BLOCK):
+    """Grouped GEMM whose groups are given by prefix sums of their row counts.
+
+    a uint8 [M_total, K], sfa int32 [M_total, KP], b uint8 [G, N, K],
+    sfb int32 [G, ceil(N/gran), KP], psum_m int32 [G]. Rows of group g (see
+    psum_group_rows) use B[g]; D[r] = A^[r] . B^[g]^T. Rows in no group are
+    left as they were. Returns (D float64 [M_total, N] with NaN on rows in no
+    group, valid bool [M_total]).
+    """
+    a = np.asarray(a, dtype=np.uint8)
+    b = np.asarray(b, dtype=np.uint8)
+    M_total = a.shape[0]
+    G, N, _ = b.shape
+    starts, ends = psum_group_rows(psum_m, M_total)
+    out = np.full((M_total, N), np.nan, dtype=np.float64)
+    valid = np.zeros(M_total, dtype=bool)
+    for g in range(G):
+        r0, r1 = int(starts[g]), int(ends[g])
+        if r1 <= r0:
+            continue
+        out[r0:r1] = fp8_gemm_nt(a[r0:r1], np.asarray(sfa)[r0:r1], b[g], np.asarray(sfb)[g], sfb_gran_n=sfb_gran_n)
+        valid[r0:r1] = True
+    return out, valid
 
 
 def masked_valid_rows(masked_m, G: int, max_m: int) -> np.ndarray:

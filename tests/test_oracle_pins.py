@@ -736,3 +736,106 @@ def _planted_rows(kind):
 @pytest.mark.parametrize("kind", ["block_index", "next_row", "first_row"])
 def test_per_row_pins_catch_planted_mistakes(kind):
     assert not one_hot_check(_planted_rows(kind), gran=1), kind
+
+
+# ------------------------------------------- groups given by psum_m ----
+# Reading of "DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs",
+# Tensor-Based Metadata Arguments: psum_m[g] is the inclusive prefix sum of the
+# groups' row counts; group g owns rows [psum_m[g-1], psum_m[g]) of A.
+
+def test_psum_rows_hand_worked():
+    # well formed: counts 2, 0, 4 over 7 rows (row 6 in no group)
+    s, e = oracle.psum_group_rows([2, 2, 6], 7)
+    assert list(s) == [0, 2, 2] and list(e) == [2, 2, 6]
+    # malformed entries: negative, decreasing, past M_total
+    s, e = oracle.psum_group_rows([-3, 5, 2, 9, 100], 8)
+    assert list(s) == [0, 0, 5, 5, 8] and list(e) == [0, 5, 5, 8, 8]
+
+
+def _psum_exact(a, ea, b, eb, owner):
+    """Exact rational D for rows with an owning group (owner[r] = g or -1), 128x128 B blocks."""
+    M, K = a.shape
+    N = b.shape[1]
+    av, bv = torch_e4m3(a), [torch_e4m3(b[g]) for g in range(b.shape[0])]
+    out = {}
+    for r in range(M):
+        g = owner[r]
+        if g < 0:
+            continue
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                acc += (Fraction(av[r, k]) * Fraction(2) ** (int(ea[r, k // 128]) - 127) *
+                        Fraction(bv[g][n, k]) * Fraction(2) ** (int(eb[g, n // 128, k // 128]) - 127))
+            out[(r, n)] = acc
+    return out
+
+
+def test_psum_equals_exact_rational_brute_force():
+    rng = np.random.default_rng(31)
+    M, N, K, G = 7, 3, 256, 3
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (G, N, K))
+    ea = rng.integers(124, 131, size=(M, 2)).astype(np.uint8)
+    eb = rng.integers(124, 131, size=(G, 1, 2)).astype(np.uint8)
+    psum = [2, 2, 6]
+    owner = [0, 0, 2, 2, 2, 2, -1]  # written out by hand from the reading
+    d, valid = oracle.m_grouped_fp8_gemm_nt_psum(a, _pack_bytes(ea), b,
+                                                 _pack_bytes(eb.reshape(G, 2)).reshape(G, 1, 1), psum)
+    exact = _psum_exact(a, ea, b, eb, owner)
+    assert list(valid) == [o >= 0 for o in owner]
+    assert np.all(np.isnan(d[6]))
+    for (r, n), v in exact.items():
+        assert Fraction(d[r, n]) == v, (r, n)
+
+
+def test_psum_reduces_to_the_contiguous_form():
+    # the same rows tagged per row with their group (m_indices) give the same D
+    rng = np.random.default_rng(32)
+    M, N, K, G = 300, 140, 384, 4
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (G, N, K))
+    sfa = _pack_bytes(rng.integers(122, 133, size=(M, K // 128)).astype(np.uint8))
+    sfb = _pack_bytes(rng.integers(120, 136, size=(G * 2, K // 128)).astype(np.uint8)).reshape(G, 2, -1)
+    counts = [37, 0, 150, 90]  # 277 rows in groups, 23 in none
+    psum = np.cumsum(counts)
+    m_indices = np.concatenate([np.full(c, g) for g, c in enumerate(counts)] + [np.full(M - psum[-1], -1)])
+    d, valid = oracle.m_grouped_fp8_gemm_nt_psum(a, sfa, b, sfb, psum)
+    dc, vc = oracle.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices.astype(np.int32))
+    assert np.array_equal(valid, vc)
+    assert np.array_equal(d[valid], dc[vc])
+
+
+def _planted_psum(kind):
+    """A copy of the psum oracle with one plausible mistake planted (CPU only)."""
+    def fn(a, sfa, b, sfb, psum_m):
+        M = a.shape[0]
+        ps = np.asarray(psum_m, dtype=np.int64)
+        if kind == "exclusive_read":       # psum_m taken as the groups' first rows
+            starts, ends = ps, np.concatenate([ps[1:], [M]])
+        elif kind == "no_running_max":     # decreasing entries not clamped
+            ends = np.minimum(np.maximum(ps, 0), M)
+            starts = np.concatenate([[0], ends[:-1]])
+        else:                              # "expert_off_by_one": group g uses B[g + 1]
+            starts, ends = oracle.psum_group_rows(ps, M)
+        out = np.full((M, b.shape[1]), np.nan)
+        for g in range(b.shape[0]):
+            if ends[g] > starts[g]:
+                gb = min(g + 1, b.shape[0] - 1) if kind == "expert_off_by_one" else g
+                out[starts[g]:ends[g]] = oracle.fp8_gemm_nt(a[starts[g]:ends[g]], sfa[starts[g]:ends[g]], b[gb], sfb[gb])
+        return out
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["exclusive_read", "no_running_max", "expert_off_by_one"])
+def test_psum_pins_catch_planted_mistakes(kind):
+    rng = np.random.default_rng(33)
+    M, N, K, G = 40, 16, 128, 4
+    a = _rand_codes(rng, (M, K))
+    b = _rand_codes(rng, (G, N, K))
+    sfa = _pack_bytes(np.full((M, 1), 127, np.uint8))
+    sfb = _pack_bytes(np.full((G, 1), 127, np.uint8)).reshape(G, 1, 1)
+    psum = np.array([10, 25, 20, 38])  # one decreasing entry: group 2 is empty
+    want, _ = oracle.m_grouped_fp8_gemm_nt_psum(a, sfa, b, sfb, psum)
+    got = _planted_psum(kind)(a, sfa, b, sfb, psum)
+    assert not np.array_equal(np.nan_to_num(got, nan=1e300), np.nan_to_num(want, nan=1e300)), kind
