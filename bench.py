@@ -336,6 +336,27 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                      "valid_rows": rows, "M_total": p["M_total"]}
     del p, sfa, sfb, d
 
+    # the same experts and row counts without padding, groups given by psum_m
+    p = W.psum_t(W.contiguous_counts(), 4096, 7168, seed=1002, device=dev)
+    sfa = dg.pack_ue8m0(p["sfa_f32"])
+    sfb = dg.pack_ue8m0(p["sfb_f32"])
+    d = torch.empty((p["M_total"], p["N"]), dtype=torch.bfloat16, device=dev)
+    op = lambda: dg.m_grouped_fp8_gemm_nt_psum(p["a"], sfa, p["b"], sfb, d, p["psum_m"])
+    op()
+    g = EventGraph([op] * reps)
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.median(g.durations_ms())
+    g.close()
+    rows = p["M_total"]
+    fl = gemm_flops(rows, p["N"], p["K"])
+    kp = kp_of(p["K"])
+    by = rows * p["K"] + p["G"] * p["N"] * p["K"] + 2 * rows * p["N"] + 4 * rows * kp + \
+        4 * p["G"] * (p["N"] // 128) * kp + 4 * p["G"]
+    out["psum_8x4096x7168"] = {"us": ms * 1e3, "TFLOP/s": fl / ms / 1e9, "GB/s": by / ms / 1e6,
+                               "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor", "rows": rows}
+    del p, sfa, sfb, d
+
     def masked_case(name, p, with_pack, rng):
         G, max_m, N, K = p["G"], p["max_m"], p["N"], p["K"]
         kp = kp_of(K)

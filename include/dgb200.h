@@ -271,6 +271,32 @@ DG_API dg_status m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa,
                                        int G, int max_m, int N, int K, void* stream);
 
 /*
+ * M-grouped FP8 GEMM with the groups given by psum_m ("DeepGEMM CUDA Graph
+ * Compatibility for Masked Grouped GEMMs", Tensor-Based Metadata Arguments:
+ * psum_m is passed as a pre-allocated device tensor; the page gives no
+ * definition). Reading: psum_m[g] is the inclusive prefix sum of the groups'
+ * row counts, so the rows of all groups lie end to end in A without padding
+ * and group g owns rows [psum_m[g-1], psum_m[g]) (psum_m[-1] = 0).
+ *   a       : device, E4M3 [M_total, K]
+ *   sfa     : device, int32 [M_total, KP]
+ *   b       : device, E4M3 [G, N, K]
+ *   sfb     : device, int32 [G, ceil(N/128), KP]
+ *   d       : device, bf16 [M_total, N]
+ *   psum_m  : device, int32 [G], read on the device only.
+ * On the device the group ends are clamped to a running maximum in
+ * [0, M_total] (end_g = min(max(0, psum_m[0..g]), M_total), start_g =
+ * end_{g-1}): a decreasing entry gives an empty group, no row belongs to two
+ * groups, and rows in no group (past the last end) are never written.
+ * A group may start at any row: a 128-row tile that reaches into the next
+ * group computes those rows but writes only its own. Limits as the masked
+ * form (G <= 1024); single CTAs. The grid depends only on (M_total, N, K, G),
+ * so a captured graph can be replayed with new psum_m.
+ */
+DG_API dg_status m_grouped_fp8_gemm_nt_psum(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                                            void* d, const int32_t* psum_m, int M_total, int N, int K, int G,
+                                            void* stream);
+
+/*
  * The three FP8 forms with a choice of B-scale granularity ("DeepInside
  * DeepGEMM", section 4: the minimal FP8 GEMM example gives the right-hand
  * operand one scale row per row, b_sf of shape [n, k / 128]).

@@ -27,6 +27,7 @@ __all__ = [
     "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc", "quantize_fp8_1x128",
     "fp8_gemm_nn", "fp8_gemm_tn", "fp8_gemm_tt",
     "fp8_gemm_nt_sfb_gran", "m_grouped_fp8_gemm_nt_contiguous_sfb_gran", "m_grouped_fp8_gemm_nt_masked_sfb_gran",
+    "m_grouped_fp8_gemm_nt_psum",
     "DEVERR_TIMEOUT", "DEVERR_MIXED_EXPERT_BLOCK",
 ]
 
@@ -102,6 +103,8 @@ def load():
         L.m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_masked.restype = i32
         L.m_grouped_fp8_gemm_nt_masked.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+        L.m_grouped_fp8_gemm_nt_psum.restype = i32
+        L.m_grouped_fp8_gemm_nt_psum.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
         L.fp8_gemm_nt_sfb_gran.restype = i32
         L.fp8_gemm_nt_sfb_gran.argtypes = [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, vp]
         L.m_grouped_fp8_gemm_nt_contiguous_sfb_gran.restype = i32
@@ -307,6 +310,24 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, d, masked_m, max_m=None):
     _check("m_grouped_fp8_gemm_nt_masked",
            load().m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m),
                                                G, max_m, N, K, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_psum(a, sfa, b, sfb, d, psum_m):
+    """M-grouped GEMM with groups given by psum_m (device int32 [G]): group g owns
+    rows [psum_m[g-1], psum_m[g]) of a [M_total, K]; rows in no group are not written."""
+    _need(a, "a", _FP8)
+    M_total, K = a.shape
+    _need(b, "b", _FP8)
+    G, N = b.shape[0], b.shape[1]
+    _need(b, "b", _FP8, (G, N, K))
+    _need(sfa, "sfa", _I32, (M_total, _kp(K)))
+    _need(sfb, "sfb", _I32, (G, (N + BLOCK - 1) // BLOCK, _kp(K)))
+    _need(d, "d", _BF16, (M_total, N))
+    _need(psum_m, "psum_m", _I32, (G,))
+    _check("m_grouped_fp8_gemm_nt_psum",
+           load().m_grouped_fp8_gemm_nt_psum(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(psum_m),
+                                             M_total, N, K, G, _stream()))
     return d
 
 

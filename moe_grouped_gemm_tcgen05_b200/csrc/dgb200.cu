@@ -127,7 +127,8 @@ struct KernelEntry {
 #define DG_LAYOUT(BN, LAYOUT) DG_ENTRY_TL(BN, dg::kDense, 1, dg::kE4M3, LAYOUT)
 #define DG_ENTRY(BN, KIND, CG) DG_ENTRY_T(BN, KIND, CG, dg::kE4M3)
 #define DG_BF16_MASKED(BN) DG_ENTRY_T(BN, dg::kMasked, 1, dg::kBF16)
-#define DG_ALL_KINDS(BN) DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1)
+#define DG_ALL_KINDS(BN) \
+    DG_ENTRY(BN, dg::kDense, 1), DG_ENTRY(BN, dg::kContiguous, 1), DG_ENTRY(BN, dg::kMasked, 1), DG_ENTRY(BN, dg::kPsum, 1)
 
 const KernelEntry kKernels[] = {
     DG_ALL_KINDS(64),  DG_ALL_KINDS(96),  DG_ALL_KINDS(128), DG_ALL_KINDS(160),
@@ -361,7 +362,8 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     const int kb = k / (dt == dg::kBF16 ? 64 : 128);  // 128-byte rows of K (one pipeline stage each)
     const int kg = (kb + 3) / 4;
     const int forced_bn = g_force_bn.load();
-    const int forced_cg = kind != dg::kMasked ? g_force_cg.load() : 0;  // no pairs for the masked form
+    // no pairs for the masked and psum_m forms
+    const int forced_cg = (kind != dg::kMasked && kind != dg::kPsum) ? g_force_cg.load() : 0;
     TileChoice best{nullptr, 0, 1};
     double best_cost = 1e300;
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
@@ -647,6 +649,36 @@ dg_status masked_nt(const void* a, const int32_t* sfa, const void* b, const int3
                        static_cast<uint64_t>(G), static_cast<uint64_t>(N), static_cast<uint64_t>(G));
 }
 
+// psum_m form: A [M_total, K] with the groups' rows end to end, group g
+// owning rows [psum_m[g-1], psum_m[g]); D [M_total, N]; B [G, N, K].
+dg_status psum_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                  const int32_t* psum_m, int M_total, int N, int K, int G, void* stream) {
+    dg_status s = check_common(a, sfa, b, sfb, d, N, K);
+    if (s != DG_OK) return s;
+    if (M_total <= 0 || G <= 0 || psum_m == nullptr) return DG_ERR_INVALID_ARG;
+    if (G > dg::MAX_MASKED_GROUPS) return DG_ERR_UNSUPPORTED;
+    if (!aligned(psum_m, 4)) return DG_ERR_ALIGNMENT;
+    DeviceState* st = nullptr;
+    if ((s = current_device(&st)) != DG_OK) return s;
+    GemmParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.sfa = sfa;
+    p.sfb = sfb;
+    p.d = static_cast<__nv_bfloat16*>(d);
+    p.meta = psum_m;
+    p.rows = M_total;
+    p.n = N;
+    p.k = K;
+    p.groups = G;
+    p.num_m_blocks = (M_total + dg::BM - 1) / dg::BM;
+    // a group boundary inside a 128-row block adds at most one block per group
+    const long long mb_total = static_cast<long long>(p.num_m_blocks) + G;
+    const long long bytes = static_cast<long long>(M_total) * K + static_cast<long long>(G) * N * K +
+                            2LL * M_total * N;
+    return launch_gemm(dg::kPsum, p, mb_total, mb_total, bytes, stream, st, a, b, 2, 3,
+                       static_cast<uint64_t>(M_total), 1, static_cast<uint64_t>(N), static_cast<uint64_t>(G));
+}
+
 }  // namespace
 
 extern "C" {
@@ -852,6 +884,11 @@ dg_status m_grouped_fp8_gemm_nt_masked_sfb_gran(const void* a, const int32_t* sf
     const dg_status s = sfb_granularity(sfb_gran_n, &per_row);
     if (s != DG_OK) return s;
     return masked_nt(a, sfa, b, sfb, per_row, d, masked_m, G, max_m, N, K, stream);
+}
+
+dg_status m_grouped_fp8_gemm_nt_psum(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                                     const int32_t* psum_m, int M_total, int N, int K, int G, void* stream) {
+    return psum_nt(a, sfa, b, sfb, d, psum_m, M_total, N, K, G, stream);
 }
 
 dg_status m_grouped_bf16_gemm_nt_masked(const void* a, const void* b, void* d, const int32_t* masked_m, int G,

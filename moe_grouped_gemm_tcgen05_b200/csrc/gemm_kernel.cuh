@@ -68,7 +68,9 @@
 
 namespace dg {
 
-enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+// kPsum: groups given by psum_m, the inclusive prefix sums of their row counts
+// (group g owns rows [psum_m[g-1], psum_m[g]) of an unpadded A).
+enum GemmKind : int { kDense = 0, kContiguous = 1, kMasked = 2, kPsum = 3 };
 // Operand type: E4M3 with packed UE8M0 block scales, or plain BF16 (no scales).
 enum OperandType : int { kE4M3 = 0, kBF16 = 1 };
 
@@ -126,7 +128,8 @@ struct GemmParams {
 // block; dense: none).
 template <int KIND>
 __host__ __device__ constexpr int sched_ints() {
-    return KIND == kMasked ? 2 * MAX_MASKED_GROUPS + 8 : (KIND == kContiguous ? MAX_CACHED_BLOCKS + 8 : 16);
+    return (KIND == kMasked || KIND == kPsum) ? 2 * MAX_MASKED_GROUPS + 8
+                                             : (KIND == kContiguous ? MAX_CACHED_BLOCKS + 8 : 16);
 }
 
 template <int BN, int CG, int SCHED_INTS, int DT = kE4M3>
@@ -172,6 +175,7 @@ struct Tile {
     int kg0, kg1;             // K groups [kg0, kg1) of this work unit
     int base, split;          // output tile index and split index (split-K; else base = t, split = 0)
     int e_own[2];             // contiguous: expert of each CTA's 128-row block (-1: padding only)
+    int row0;                 // psum_m form: first row of A (and D) of the tile
 };
 
 // ----------------------------------------------------------------- waits ----
@@ -244,19 +248,30 @@ __device__ __forceinline__ bool raster_tile(const GemmParams& p, int t_unit, Til
     return true;
 }
 
-// Masked: tiles of group g are numbered from s_prefix[g]; within a group the
-// m-block varies fastest. `gcur` is the caller's monotone cursor.
+// Rows of group g. Masked: s_mm[g] is the clamped masked_m. psum_m form: s_mm
+// holds the groups' first rows (g = 0..groups), so group g has s_mm[g+1] - s_mm[g].
+template <int KIND>
+__device__ __forceinline__ int group_rows(const int* s_mm, int g) {
+    if constexpr (KIND == kPsum) return s_mm[g + 1] - s_mm[g];
+    else return s_mm[g];
+}
+
+// Masked and psum_m forms: tiles of group g are numbered from s_prefix[g];
+// within a group the m-block varies fastest. `gcur` is the caller's monotone
+// cursor.
+template <int KIND>
 __device__ __forceinline__ bool masked_tile(const int* s_prefix, const int* s_mm, int groups, int t, int& gcur,
                                             Tile& c) {
     if (t >= s_prefix[groups]) return false;
     while (s_prefix[gcur + 1] <= t) ++gcur;
     const int local = t - s_prefix[gcur];
-    const int mb = (s_mm[gcur] + BM - 1) / BM;
+    const int mb = (group_rows<KIND>(s_mm, gcur) + BM - 1) / BM;
     c.g = gcur;
     c.n_blk = local / mb;
     c.m_blk = local - c.n_blk * mb;
     c.base = t;
     c.split = 0;
+    c.row0 = (KIND == kPsum ? s_mm[gcur] : 0) + c.m_blk * BM;
     return true;
 }
 
@@ -294,10 +309,10 @@ __device__ __forceinline__ int cached_block_expert(const GemmParams& p, const in
 template <int KIND, bool NEED_EXPERT, int CG>
 __device__ __forceinline__ bool next_tile(const GemmParams& p, const int* s_prefix, const int* s_mm, int& t,
                                           int units, int& gcur, Tile& c, uint32_t lane) {
-    if constexpr (KIND == kMasked) {
+    if constexpr (KIND == kMasked || KIND == kPsum) {
         c.kg0 = 0;
         c.kg1 = (p.kb + 3) / 4;
-        return masked_tile(s_prefix, s_mm, p.groups, t, gcur, c);
+        return masked_tile<KIND>(s_prefix, s_mm, p.groups, t, gcur, c);
     } else if constexpr (KIND == kContiguous && CG == 2) {
         const int per_pass = p.num_m_blocks * p.num_n_blocks;
         for (; t < 2 * per_pass; t += units) {
@@ -465,7 +480,7 @@ struct ScaleQuads {
 // EPI 0: plain bf16 D.
 template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
-    static_assert(CG == 1 || KIND != kMasked, "CTA pairs are built for the dense and contiguous forms");
+    static_assert(CG == 1 || (KIND != kMasked && KIND != kPsum), "CTA pairs are built for the dense and contiguous forms");
     static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
     static_assert(LAYOUT == 0 || (KIND == kDense && CG == 1 && DT == kE4M3), "layouts: dense, single CTAs");
     static_assert(!(LAYOUT & 2) || BN % 128 == 0, "an MN-major B tile is whole 128-byte atoms");
@@ -507,8 +522,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);  // split-K: this unit reduces
-    int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked)
-    int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups]     (masked)
+    int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked, psum_m)
+    int* s_mm = s_prefix + MAX_MASKED_GROUPS + 4;                   // [groups] (masked), [groups + 1] (psum_m)
     int* s_bexp = s_prefix;                                          // [128-row blocks] (contiguous)
 
     const uint32_t warp = threadIdx.x / 32;
@@ -552,16 +567,48 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     griddep_wait();
     griddep_launch_dependents();
     if constexpr (KIND == kMasked) {
-        // masked_m clamped to [0, max_m]; tile prefix over groups (warp 0 scans).
+        // masked_m clamped to [0, max_m]
         for (int g = threadIdx.x; g < p.groups; g += NUM_THREADS) s_mm[g] = min(max(__ldg(p.meta + g), 0), p.rows);
         __syncthreads();
+    }
+    if constexpr (KIND == kPsum) {
+        // first row of every group: s_mm[0] = 0, s_mm[g + 1] = end of group g =
+        // min(max(0, psum_m[0..g]), M_total), a running max so that no row
+        // belongs to two groups (warp 0: per-lane maxima, then a max-scan)
+        if (warp == 0) {
+            const int per = (p.groups + 31) / 32;
+            const int g0 = static_cast<int>(lane) * per;
+            int mx = 0;
+            for (int i = 0; i < per; ++i)
+                if (g0 + i < p.groups) mx = max(mx, __ldg(p.meta + g0 + i));
+            int incl = mx;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= static_cast<uint32_t>(o)) incl = max(incl, v);
+            }
+            int run = __shfl_up_sync(0xffffffffu, incl, 1);
+            if (lane == 0) run = 0;
+            for (int i = 0; i < per; ++i) {
+                const int g = g0 + i;
+                if (g < p.groups) {
+                    run = max(run, __ldg(p.meta + g));
+                    s_mm[g + 1] = min(run, p.rows);
+                }
+            }
+            if (lane == 0) s_mm[0] = 0;
+        }
+        __syncthreads();
+    }
+    if constexpr (KIND == kMasked || KIND == kPsum) {
+        // tile prefix over groups (warp 0 scans)
         if (warp == 0) {
             const int per = (p.groups + 31) / 32;
             const int g0 = static_cast<int>(lane) * per;
             int sum = 0;
             for (int i = 0; i < per; ++i) {
                 const int g = g0 + i;
-                if (g < p.groups) sum += ((s_mm[g] + BM - 1) / BM) * p.num_n_blocks;
+                if (g < p.groups) sum += ((group_rows<KIND>(s_mm, g) + BM - 1) / BM) * p.num_n_blocks;
             }
             int incl = sum;
 #pragma unroll
@@ -574,7 +621,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 const int g = g0 + i;
                 if (g < p.groups) {
                     s_prefix[g] = run;
-                    run += ((s_mm[g] + BM - 1) / BM) * p.num_n_blocks;
+                    run += ((group_rows<KIND>(s_mm, g) + BM - 1) / BM) * p.num_n_blocks;
                 }
             }
             if (lane == 31) s_prefix[p.groups] = incl;
@@ -636,7 +683,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         bool aborted = false;
         for (int t = unit; !aborted && next_tile<KIND, true, CG>(p, s_prefix, s_mm, t, units, gcur, cur, lane);
              t += units) {
-            const int a_row = cur.m_blk * BM * CG + my_rows;
+            const int a_row = (KIND == kPsum ? cur.row0 : cur.m_blk * BM * CG) + my_rows;
             const int b_row = cur.n_blk * BN + Cfg::B_ROWS * static_cast<int>(rank);
             const int g = max(cur.g, 0);
             for (int gi = cur.kg0; gi < cur.kg1 && !aborted; ++gi) {
@@ -714,7 +761,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             int ckg = cok ? ctile.kg0 : 0;
             auto load_next = [&](ScaleWords<BN, KIND, CG>& w) -> bool {
                 if (!cok) return false;
-                w.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, rot_group(p, ct, ckg, kg_count), lane);
+                w.load(p, KIND == kPsum ? ctile.row0 : ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g,
+                       rot_group(p, ct, ckg, kg_count), lane);
                 if (++ckg == ctile.kg1) {
                     ct += units;
                     cok = next_tile<KIND, true, CG>(p, s_prefix, s_mm, ct, units, cg_cur, ctile, lane);
@@ -756,7 +804,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     if (!cok) return false;
                     q.lo = max(q_base, ctile.kg0);
                     q.hi = min(q_base + 4, ctile.kg1);
-                    q.load(p, ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, q_base, lane);
+                    q.load(p, KIND == kPsum ? ctile.row0 : ctile.m_blk * BM * CG, ctile.n_blk * BN, ctile.g, q_base,
+                           lane);
                     q_base += 4;
                     if (q_base >= ctile.kg1) {
                         ct += units;
@@ -947,6 +996,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             } else if constexpr (KIND == kMasked) {
                 valid = mloc < s_mm[c.g];
                 out_row = static_cast<size_t>(c.g) * p.rows + mloc;
+            } else if constexpr (KIND == kPsum) {
+                valid = mloc < group_rows<kPsum>(s_mm, c.g);   // mloc counts from the group's first row
+                out_row = static_cast<size_t>(s_mm[c.g] + mloc);
             } else {
                 const int id = (mloc < p.rows) ? __ldg(p.meta + mloc) : -1;
                 const bool in_range = id >= 0 && id < p.groups;
@@ -1090,6 +1142,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     __syncwarp();
                     if (lane == 0) {
                         if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
+                        else if constexpr (KIND == kPsum) tma_store_2d(&p.tma_d, sb, col, s_mm[c.g] + row_coord);
                         else tma_store_2d(&p.tma_d, sb, col, row_coord);
                         bulk_commit_group();
                     }

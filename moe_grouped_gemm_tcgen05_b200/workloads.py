@@ -143,6 +143,26 @@ def contiguous(counts, N: int, K: int, seed: int, align: int = BLOCK, tail_block
                 M_total=M_total, N=N, K=K, G=G)
 
 
+def psum(counts, M_total: int, N: int, K: int, seed: int, sfb_gran_n: int = BLOCK):
+    """Grouped problem with the groups given by psum_m: group g owns counts[g]
+    rows, the groups' rows end to end from row 0 without padding; psum_m is
+    the running total of counts. Rows past sum(counts) (up to M_total) belong
+    to no group and hold NaN bytes."""
+    rng = rng_for(seed)
+    counts = np.asarray(counts, dtype=np.int64)
+    G = counts.shape[0]
+    used = int(counts.sum())
+    assert used <= M_total
+    a = np.full((M_total, K), NAN_BYTE, dtype=np.uint8)
+    sfa = np.ones((M_total, K // BLOCK), dtype=np.float32)
+    qa, qs = quantise_rows(_normal(rng, (used, K)))
+    a[:used] = qa
+    sfa[:used] = qs
+    b, sfb = grouped_weights(rng, G, N, K, sfb_gran_n)
+    psum_m = np.cumsum(counts).astype(np.int32)
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, psum_m=psum_m, M_total=M_total, N=N, K=K, G=G)
+
+
 def masked(masked_m, max_m: int, N: int, K: int, seed: int, fill_invalid_nan: bool = True,
            sfb_gran_n: int = BLOCK):
     """Masked M-grouped problem: a [G,max_m,K], b [G,N,K]; rows >= masked_m hold NaN bytes."""
@@ -304,6 +324,17 @@ def contiguous_t(counts, N: int, K: int, seed: int, align: int = BLOCK, device="
     b, sfb = grouped_weights_t(g, G, N, K, device)
     m_indices = torch.from_numpy(mi).to(device)
     return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, m_indices=m_indices, M_total=M_total, N=N, K=K, G=G)
+
+
+def psum_t(counts, N: int, K: int, seed: int, device="cuda"):
+    """psum on the device: the groups' rows end to end (M_total = sum(counts))."""
+    G = len(counts)
+    M_total = int(sum(int(c) for c in counts))
+    g = _gen(device, seed)
+    a, sfa = quantise_rows_t(torch.randn((M_total, K), generator=g, device=device))
+    b, sfb = grouped_weights_t(g, G, N, K, device)
+    psum_m = torch.from_numpy(np.cumsum(np.asarray(counts, dtype=np.int64)).astype(np.int32)).to(device)
+    return dict(a=a, sfa_f32=sfa, b=b, sfb_f32=sfb, psum_m=psum_m, M_total=M_total, N=N, K=K, G=G)
 
 
 def masked_t(masked_m, max_m: int, N: int, K: int, seed: int, device="cuda"):
