@@ -6,15 +6,18 @@
  * CUDA device; `stream` is a cudaStream_t passed as void* (NULL = legacy
  * default stream).
  *
- * Operation (all three GEMM forms): D = A . B^T ("NT"), E4M3 operands, fp32
- * accumulation, bf16 output, no C term. Sources: "DeepInside DeepGEMM:
+ * Operation (dense, contiguous, masked and psum_m GEMM forms): D = A . B^T
+ * ("NT"), E4M3 operands, fp32 accumulation, bf16 output, no C term (the
+ * C term, fp32 output, other operand layouts and BF16 operands have calls of
+ * their own below). Sources: "DeepInside DeepGEMM:
  * Unpacking DeepSeek's Unified Tensor Core Library for SM90 and SM100",
  * section 4 (the standard non-grouped FP8 NT GEMM computes D = C + A @ B.T)
  * and section 2 (on SM100 the scaling factors are UE8M0, four packed into one
  * torch.int).
  *
  * Scales. Activations (A) carry one scale per 1x128 block along K, weights (B)
- * one scale per 128x128 block. A scale is a UE8M0 byte e meaning 2^(e-127).
+ * one scale per 128x128 block (the *_sfb_gran calls also take one per 1x128
+ * block of each row of B). A scale is a UE8M0 byte e meaning 2^(e-127).
  * Scale rows are packed four bytes per int32, little-endian, consecutive
  * along K: byte j of word i is K-block 4*i + j. With KB = K/128 and
  * KP = ceil(KB/4):
@@ -33,7 +36,7 @@
  * configuration fixed by the scalar sizes alone ("DeepGEMM CUDA Graph
  * Compatibility for Masked Grouped GEMMs: Implementation Guide", sections
  * Stateless Kernel Architecture and Tensor-Based Metadata Arguments). All
- * variable metadata (masked_m, m_indices, scales) is read on the device. The
+ * variable metadata (masked_m, psum_m, m_indices, scales) is read on the device. The
  * first call on a device configures the kernels (cudaFuncSetAttribute); make
  * it, or dgb200_init(), before capturing.
  *
@@ -48,7 +51,7 @@
  * hanging.
  *
  * Limits: 1 <= M, N; N % 8 == 0; K % 128 == 0; 128 <= K <= 2^20;
- * rows * K < 2^40 for every operand; G <= 1024 for the masked form.
+ * rows * K < 2^40 for every operand; G <= 1024 for the masked and psum_m forms.
  */
 #ifndef DGB200_H
 #define DGB200_H

@@ -1,11 +1,12 @@
 // Persistent, warp-specialised FP8 block-scaled GEMM for sm_100a.
 //
 // D = A . B^T with E4M3 operands, packed UE8M0 scales (one per 1x128 block of
-// A, one per 128x128 block of B), fp32 accumulation in TMEM, bf16 output. One
-// template serves the three forms of the method ("DeepInside DeepGEMM" section
-// 4 for the dense NT GEMM; "DeepGEMM CUDA Graph Compatibility for Masked
-// Grouped GEMMs" for the masked form; the contiguous form is the "continuous
-// storage layout" of "DeepGEMM tested by Novita AI").
+// A, one per 128x128 block of B or one per 1x128 block of each row of B),
+// fp32 accumulation in TMEM, bf16 output. One template serves the forms of the
+// method ("DeepInside DeepGEMM" section 4 for the dense NT GEMM; "DeepGEMM CUDA
+// Graph Compatibility for Masked Grouped GEMMs" for the masked form and for
+// the groups given by psum_m; the contiguous form is the "continuous storage
+// layout" of "DeepGEMM tested by Novita AI"), and also the BF16 masked GEMM.
 //
 // CTA = 7 warps, one CTA per SM, persistent over a grid fixed by the sizes:
 //   warp 0      TMA producer: loads of the A and B tiles (128-byte swizzle)
@@ -25,8 +26,8 @@
 //               fp32 -> bf16 with round-to-nearest-even, 32x32 chunks staged
 //               in swizzled shared memory and written by TMA; chunks holding
 //               rows that must not be written (past masked_m, padding of
-//               m_indices) use predicated row stores instead, so those rows
-//               are never touched.
+//               m_indices, past a psum_m group's end) use predicated row
+//               stores instead, so those rows are never touched.
 // Every role runs its loop on the whole warp: waits are warp-wide votes and
 // the TMA / tcgen05 instructions are issued by one lane chosen with
 // elect.sync. (A loop run by one lane, or guarded by a lane test, leaves the
@@ -87,15 +88,15 @@ constexpr uint32_t DEVERR_TIMEOUT = 1u;
 constexpr uint32_t DEVERR_MIXED_EXPERT_BLOCK = 2u;
 
 struct GemmParams {
-    CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous) or 3-D {K, max_m, G} (masked)
+    CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous, psum_m) or 3-D {K, max_m, G} (masked)
     CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped); box BN/CG rows
     CUtensorMap tma_d;        // D (bf16, store): 2-D {N, rows} or 3-D {N, max_m, G}; 32x32 box, 64-byte swizzle
     const int32_t* sfa;       // packed scale rows of A
     const int32_t* sfb;       // packed scale rows of B (per 128 rows or per row, per group)
     __nv_bfloat16* d;         // output
-    const int32_t* meta;      // m_indices (contiguous) / masked_m (masked) / null
+    const int32_t* meta;      // m_indices (contiguous) / masked_m (masked) / psum_m (psum_m) / null
     uint32_t* status;         // device status word
-    int rows;                 // M (dense), M_total (contiguous), max_m (masked)
+    int rows;                 // M (dense), M_total (contiguous, psum_m), max_m (masked)
     int n, k, groups;
     int kb;                   // K / 128
     int kp;                   // ceil(kb / 4) packed words per scale row
@@ -124,8 +125,8 @@ struct GemmParams {
 };
 
 // SCHED_INTS: 32-bit words of shared memory for the tile scheduler (masked:
-// clamped masked_m and tile prefix sums; contiguous: expert of every 128-row
-// block; dense: none).
+// clamped masked_m and tile prefix sums; psum_m: the groups' first rows and
+// tile prefix sums; contiguous: expert of every 128-row block; dense: none).
 template <int KIND>
 __host__ __device__ constexpr int sched_ints() {
     return (KIND == kMasked || KIND == kPsum) ? 2 * MAX_MASKED_GROUPS + 8
@@ -171,7 +172,7 @@ struct GemmConfig {
 };
 
 struct Tile {
-    int m_blk, n_blk, g;      // g: group (masked) or expert (contiguous), 0 for dense
+    int m_blk, n_blk, g;      // g: group (masked, psum_m) or expert (contiguous), 0 for dense
     int kg0, kg1;             // K groups [kg0, kg1) of this work unit
     int base, split;          // output tile index and split index (split-K; else base = t, split = 0)
     int e_own[2];             // contiguous: expert of each CTA's 128-row block (-1: padding only)
