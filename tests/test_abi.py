@@ -88,6 +88,14 @@ def test_sfb_granularity_is_checked_on_the_host(lib):
     m.argtypes = [vp, vp, vp, vp, i, vp, vp, i, i, i, i, vp]
     assert m(good, good, good, good, 3, good, good, 4, 64, 128, 128, None) == 1
     assert m(good, good, good, good, 1, good, good, 2048, 64, 128, 128, None) == 3    # too many groups
+    ps = lib.m_grouped_fp8_gemm_nt_psum
+    ps.restype = i
+    ps.argtypes = [vp] * 6 + [i] * 4 + [vp]
+    assert ps(good, good, good, good, good, None, 128, 128, 128, 2, None) == 1       # null psum_m
+    assert ps(good, good, good, good, good, good, 0, 128, 128, 2, None) == 1         # M_total <= 0
+    assert ps(good, good, good, good, good, good, 128, 128, 128, 0, None) == 1       # G <= 0
+    assert ps(good, good, good, good, good, good, 128, 128, 128, 2048, None) == 3    # too many groups
+    assert ps(good, good, good, good, good, vp(0x10002), 128, 128, 128, 2, None) == 2  # psum_m alignment
     import torch
     x = torch.zeros((128, 128), dtype=torch.uint8)
     with pytest.raises(ValueError):  # the binding checks the scale-row count for the granularity

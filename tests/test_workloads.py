@@ -54,3 +54,22 @@ def test_masked_distributions():
     # closed-form mean / P(0) of the truncated Zipf(1.1) on {0..512}
     assert abs(float((m * p).sum()) - 57.4) < 0.5 and abs(p[0] - 0.191) < 0.002
     assert 30 < z.mean() < 90 and 25 < (z == 0).sum() < 75
+
+
+def test_per_row_weight_scales():
+    # one scale per 1x128 block of each row of B; rows carry a power-of-two spread
+    p = W.dense(16, 300, 512, seed=4, sfb_gran_n=1)
+    assert p["sfb_f32"].shape == (300, 4) and _is_pow2(p["sfb_f32"]).all()
+    assert np.all(np.abs(_decode(p["b"])) <= 448)
+    assert len(np.unique(p["sfb_f32"][:128, 0])) > 1  # rows of one 128-block differ
+    q = W.masked(np.array([3, 0], np.int32), 8, 136, 256, seed=5, sfb_gran_n=1)
+    assert q["sfb_f32"].shape == (2, 136, 2)
+
+
+def test_psum_layout():
+    p = W.psum([70, 0, 100], 200, 256, 512, seed=6)
+    assert list(p["psum_m"]) == [70, 70, 170] and p["psum_m"].dtype == np.int32
+    assert p["a"].shape == (200, 512) and p["b"].shape == (3, 256, 512) and p["sfb_f32"].shape == (3, 2, 4)
+    assert np.all(p["a"][170:] == W.NAN_BYTE)             # rows in no group
+    assert not np.any(p["a"][:170] == W.NAN_BYTE)
+    assert _is_pow2(p["sfa_f32"]).all()
