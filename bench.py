@@ -25,8 +25,11 @@ Also reported:
   cpu_baseline the CPU oracle (numpy float64) on a bounded sample: the first
                rows of A against all of B for each problem
   clocks       NVML SM clock and throttle reasons sampled during the timed region
-  detail       the contiguous (8 experts), masked decode (32 groups, up/down)
-               and masked Zipf (256 groups, pack + GEMM) workloads, each timed
+  detail       the contiguous (8 experts) and psum_m-grouped (the same experts
+               without padding) GEMMs, masked decode (32 groups, up/down) and
+               masked Zipf (256 groups, pack + GEMM), D = C + A.B^T in place
+               (fp32), the NN/TN/TT layouts, per-row weight scales, the
+               activation quantiser and the BF16 masked decode, each timed
                under CUDA Graph replay with per-call events (not part of value)
 
 --impl reference times the oracle as it stands on the host cores, on a bounded
