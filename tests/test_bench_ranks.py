@@ -49,3 +49,22 @@ def test_aggregate_counts_every_replica():
     one = bench.aggregate_tflops(step, 1, 0.4)
     assert abs(one - step / 0.4e-3 / 1e12) < 1e-9
     assert abs(bench.aggregate_tflops(step, 4, 0.4) - 4 * one) < 1e-9
+
+
+def test_reference_arm_under_torchrun_prints_once_from_rank_0():
+    # the launch the reference arm gets at N > 1: rank 0 alone times the
+    # oracle and prints the JSON line; the other rank exits 0 without work
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()),
+           "bench.py", "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["e2e"]["h2d_bytes_per_step"] == 0
