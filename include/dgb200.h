@@ -29,7 +29,14 @@
  * K bytes, D rows N bf16 values.
  *
  * Ownership. The caller allocates and owns every buffer. The library keeps no
- * per-call state and allocates no device memory in any call.
+ * per-call state and allocates no device memory, neither in a call nor when it
+ * sets up a device: its only device data are static variables of its module
+ * (the 4-byte status word below, and the scratch of fp8_gemm_nt_noalloc).
+ *
+ * Streams. Work goes only on the stream given. Calls are asynchronous and
+ * reentrant: calls on different streams (or host threads) may run at the same
+ * time, since no compute call except fp8_gemm_nt_noalloc touches memory other
+ * than its own arguments and the status word.
  *
  * CUDA Graph capture. Every compute entry point is capture safe: no host
  * synchronisation, no allocation, no host reads of device values, and a launch
@@ -87,12 +94,26 @@ typedef enum {
 DG_API const char* dgb200_status_string(dg_status s);
 
 /*
- * Configure the kernels for the current device: caches the SM count and sets
- * the dynamic shared-memory limits. Idempotent and thread safe. Called
- * implicitly by the first compute call on a device; call it eagerly before any
- * CUDA Graph capture.
+ * Configure the kernels for CUDA device `device` (an ordinal as in
+ * cudaSetDevice): checks that it is an sm_100 part, caches its SM count, sets
+ * the kernels' dynamic shared-memory limits and counts how many CTA pairs and
+ * clusters fit on it at once. Allocates nothing. The caller's current device
+ * is unchanged on return. Idempotent and thread safe. The first compute call
+ * on a device does the same implicitly; call this eagerly before any CUDA
+ * Graph capture.
+ * Returns DG_ERR_INVALID_ARG for an ordinal that names no device,
+ * DG_ERR_UNSUPPORTED for a device other than sm_100, DG_ERR_NOT_INITIALIZED
+ * when no CUDA driver or device is usable.
  */
-DG_API dg_status dgb200_init(void);
+DG_API dg_status dgb200_init(int device);
+
+/*
+ * Read the device status word of the current device (DG_DEVERR_* bits, 0 when
+ * no kernel recorded a problem) into *code (host pointer) and reset it to
+ * zero, like cudaGetLastError. Synchronises the device: never call it inside a
+ * stream capture.
+ */
+DG_API dg_status dgb200_last_device_error(int* code);
 
 /*
  * Read the device status word of the current device into *bits (host pointer)
@@ -121,22 +142,23 @@ DG_API int dgb200_block_n_supported(int block_n);
 DG_API dg_status dgb200_set_cta_group(int cta_group);
 
 /*
- * Split-K for the dense GEMM (process-wide; tests and tuning). 0 restores the
+ * Split-K for the dense GEMMs fp8_gemm_nt, fp8_gemm_nt_acc and
+ * fp8_gemm_nt_sfb_gran (process-wide; tests and tuning). 0 restores the
  * heuristic, which splits K only when the output tiles alone leave SMs idle
- * (small M). 1 never splits. s >= 2 splits every dense call into s ranges of
+ * (small M). 1 never splits. s >= 2 splits every such call into s ranges of
  * whole K groups (four 128-K blocks each; with G groups, range i covers groups
- * [i*G/s, (i+1)*G/s)); a combination that is not possible (s larger than G,
- * CTA pairs forced, workspace too small) makes the dense call return
- * DG_ERR_UNSUPPORTED.
- * A split unit writes its fp32 partial tile to a workspace that the library
- * allocates (40 MB, with 4096 per-tile counters) when it first sets up the
- * device. The last unit to finish a tile adds the partials in split order
- * (the same result whichever unit is last) and writes the bf16 tile. The
- * counters return to zero by themselves; after a launch that gave up
- * (DG_DEVERR_TIMEOUT), dgb200_device_error(bits, 1) zeroes them again. Calls
- * that may split must not run concurrently on two streams of one device (they
- * share the workspace).
- * Returns DG_ERR_UNSUPPORTED for s outside [0, 16].
+ * [i*G/s, (i+1)*G/s)); a combination that is not possible (s larger than G, s
+ * larger than the tile width / 8, CTA pairs forced) makes the dense call
+ * return DG_ERR_UNSUPPORTED.
+ * The s units of an output tile run as one thread-block cluster of s CTAs.
+ * Each computes the fp32 partial of its K range in tensor memory; the tile's
+ * columns are dealt out among the CTAs in 8-column pieces, every CTA sends
+ * the pieces it does not own to their owner's shared memory (distributed
+ * shared memory), and each owner adds the s partials of its pieces in split
+ * order and writes them. No global memory besides D is used, so splitting
+ * calls may run concurrently on several streams, and repeated calls give
+ * identical bits.
+ * Returns DG_ERR_UNSUPPORTED for s outside [0, 8].
  */
 DG_API dg_status dgb200_set_splits(int splits);
 
@@ -210,15 +232,21 @@ DG_API dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* 
  * synchronise the device).
  *   splits : 0 = the tile model's choice among configurations whose split-K
  *            scratch fits the static arrays below (never DG_ERR_SCRATCH_TOO_SMALL);
- *            1 = no split-K; s >= 2 = exactly s ranges of K groups, tiled as
- *            fp8_gemm_nt with dgb200_set_splits(s) would tile them.
- * Split-K scratch lives in file-scope __device__ arrays of the library, found
- * with cudaGetSymbolAddress: at most 8 MiB of fp32 partials (2^21 floats; a
- * split call needs ceil(M/128) * ceil(N/BN) * s * 128 * BN * 4 bytes for its N
- * tile BN) and 1024 output tiles. A request beyond either limit returns
- * DG_ERR_SCRATCH_TOO_SMALL before any device work; s > 16 returns
- * DG_ERR_UNSUPPORTED. A splitting call first zeroes the tile counters it uses
- * (an asynchronous memset on `stream`).
+ *            1 = no split-K; s >= 2 = exactly s ranges of K groups (as
+ *            dgb200_set_splits describes), with the tile width chosen among
+ *            those whose partials fit the static arrays.
+ * Unlike the other dense calls, the units of a split tile here meet through
+ * global scratch, not inside a cluster: each writes its fp32 partial tile to
+ * the scratch and the last one to finish adds the partials in split order
+ * (the same order as the cluster form, so equal configurations give equal
+ * bits). The scratch lives in file-scope __device__ arrays of the library,
+ * found with cudaGetSymbolAddress: at most 8 MiB of fp32 partials (2^21
+ * floats; a split call needs ceil(M/128) * ceil(N/BN) * s * 128 * BN * 4 bytes
+ * for its N tile BN) and 1024 output tiles. A request that no tile width can
+ * serve within these limits returns DG_ERR_SCRATCH_TOO_SMALL before any device
+ * work;
+ * s > 16 returns DG_ERR_UNSUPPORTED. A splitting call first zeroes the tile
+ * counters it uses (an asynchronous memset on `stream`).
  * The scratch is shared by every caller of this function on a device: calls
  * that overlap in time (two streams, two host threads, or one call still
  * running when the next one starts on another stream) race on it and give

@@ -21,7 +21,7 @@ import threading
 import torch
 
 __all__ = [
-    "BLOCK", "lib_path", "load", "init", "device_error", "set_block_n", "block_n_supported",
+    "BLOCK", "lib_path", "load", "init", "device_error", "last_device_error", "set_block_n", "block_n_supported",
     "fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
     "pack_ue8m0", "pack_ue8m0_validate", "DgError", "set_test_hooks", "set_cta_group", "set_splits",
     "fp8_gemm_nt_noalloc", "m_grouped_bf16_gemm_nt_masked", "fp8_gemm_nt_acc", "quantize_fp8_1x128",
@@ -73,7 +73,9 @@ def load():
         L.dgb200_status_string.restype = ctypes.c_char_p
         L.dgb200_status_string.argtypes = [i32]
         L.dgb200_init.restype = i32
-        L.dgb200_init.argtypes = []
+        L.dgb200_init.argtypes = [i32]
+        L.dgb200_last_device_error.restype = i32
+        L.dgb200_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_int)]
         L.dgb200_device_error.restype = i32
         L.dgb200_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32), i32]
         L.dgb200_set_block_n.restype = i32
@@ -150,9 +152,22 @@ _I32 = (torch.int32,)
 _BF16 = (torch.bfloat16,)
 
 
-def init():
-    """Configure the kernels for the current device (do it before graph capture)."""
-    _check("dgb200_init", load().dgb200_init())
+def init(device=None):
+    """Configure the kernels for a CUDA device (default: torch's current one);
+    do it before graph capture."""
+    if device is None:
+        device = torch.cuda.current_device()
+    elif isinstance(device, torch.device):
+        device = device.index if device.index is not None else torch.cuda.current_device()
+    _check("dgb200_init", load().dgb200_init(int(device)))
+
+
+def last_device_error() -> int:
+    """Device status bits (DEVERR_*) of the current device, then reset to 0;
+    synchronises the device."""
+    v = ctypes.c_int(0)
+    _check("dgb200_last_device_error", load().dgb200_last_device_error(ctypes.byref(v)))
+    return int(v.value)
 
 
 def device_error(clear: bool = True) -> int:

@@ -4,9 +4,10 @@
 // the TMA tensor maps (driver entry point, no libcuda link), picks a tile
 // width from the sizes and the SM count, and launches one kernel on the
 // caller's stream. A compute call allocates nothing, never synchronises and
-// reads no device value, so it can be captured in a CUDA Graph. Device memory
-// is allocated once per device, when the library first sets that device up:
-// the split-K workspace (partial tiles and per-tile counters).
+// reads no device value, so it can be captured in a CUDA Graph. The library
+// allocates no device memory at all: split-K adds its partial tiles inside a
+// thread-block cluster (distributed shared memory), and the device status word
+// and the scratch of fp8_gemm_nt_noalloc are static __device__ variables.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -44,18 +45,18 @@ namespace {
 using dg::GemmParams;
 
 constexpr int kMaxDevices = 64;
-
-// Split-K workspace per device: fp32 partial tiles and one counter per output
-// tile. Sized for up to two waves of 128 x 256 partials over the SMs.
-constexpr size_t kSplitWsBytes = size_t(40) << 20;
-constexpr int kSplitCounters = 4096;
+constexpr int kMaxClusterSplits = dg::MAX_CLUSTER_SPLITS;
 
 struct DeviceState {
-    bool ready = false;
+    std::atomic<bool> ready{false};  // set (release) once every field below is filled
     int sms = 0;
     uint32_t* status = nullptr;  // address of g_dg_device_status on this device
     int max_pairs[64] = {};      // co-resident CTA pairs per kernel entry (cluster kernels only)
-    float* split_ws = nullptr;   // split-K partials (null: split-K disabled on this device)
+    // co-resident clusters of s CTAs (s = 2..8) per kernel entry, for the
+    // cluster split-K of the dense single-CTA kernels (0: not launchable)
+    int max_clusters[64][kMaxClusterSplits + 1] = {};
+    // fp8_gemm_nt_noalloc only: split-K scratch in the library's static arrays
+    float* split_ws = nullptr;
     uint32_t* split_counters = nullptr;
 };
 
@@ -115,12 +116,14 @@ struct KernelEntry {
     int epi;     // dense: 1 = epilogue of D = C + A.B^T (bf16 or fp32 D)
     void* fn;
     int smem;
-    int stages;  // depth of the operand ring
+    int stages;       // depth of the operand ring
+    int stage_bytes;  // bytes of one stage (A and B tiles)
 };
 
 #define DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, EPI)                                                             \
     {BN, KIND, CG, DT, LAYOUT, EPI, kernel_ptr<BN, KIND, CG, DT, LAYOUT, EPI>(),                                \
-     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES}
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES, \
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGE_BYTES}
 #define DG_ENTRY_TL(BN, KIND, CG, DT, LAYOUT) DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, 0)
 #define DG_ENTRY_T(BN, KIND, CG, DT) DG_ENTRY_TL(BN, KIND, CG, DT, 0)
 #define DG_ACC(BN, CG) DG_ENTRY_TLE(BN, dg::kDense, CG, dg::kE4M3, 0, 1)
@@ -188,6 +191,28 @@ dg_status setup_device(int dev, DeviceState& st) {
             if (cudaOccupancyMaxActiveClusters(&clusters, e.fn, &cfg) != cudaSuccess || clusters < 1) return DG_ERR_CUDA;
             st.max_pairs[i] = clusters;
         }
+        if (e.cg == 1 && e.kind == dg::kDense && e.layout == 0 && e.dt == dg::kE4M3) {
+            // clusters of s CTAs that fit on the device at once (a cluster's CTAs share a GPC)
+            for (int s = 2; s <= kMaxClusterSplits; ++s) {
+                cudaLaunchConfig_t cfg = {};
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.gridDim = dim3(static_cast<unsigned>(s * (st.sms / s)));
+                cfg.blockDim = dim3(dg::NUM_THREADS);
+                cfg.dynamicSmemBytes = static_cast<size_t>(e.smem);
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                int clusters = 0;
+                if (cudaOccupancyMaxActiveClusters(&clusters, e.fn, &cfg) != cudaSuccess) {
+                    cudaGetLastError();
+                    clusters = 0;
+                }
+                st.max_clusters[i][s] = clusters;
+            }
+        }
     }
     void* status = nullptr;
     if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
@@ -195,27 +220,15 @@ dg_status setup_device(int dev, DeviceState& st) {
     return DG_OK;
 }
 
+// Set up device `dev`, which must be the current device. Allocates nothing.
 dg_status init_device(int dev) {
     std::lock_guard<std::mutex> lock(g_mu);
     if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
     DeviceState& st = g_dev[dev];
-    if (st.ready) return DG_OK;
+    if (st.ready.load(std::memory_order_acquire)) return DG_OK;
     const dg_status s = setup_device(dev, st);
     if (s != DG_OK) return s;
-    // split-K workspace: optional; without it the GEMMs run unsplit
-    void* ws = nullptr;
-    void* ctr = nullptr;
-    if (cudaMalloc(&ws, kSplitWsBytes) == cudaSuccess &&
-        cudaMalloc(&ctr, kSplitCounters * sizeof(uint32_t)) == cudaSuccess &&
-        cudaMemset(ctr, 0, kSplitCounters * sizeof(uint32_t)) == cudaSuccess) {
-        st.split_ws = static_cast<float*>(ws);
-        st.split_counters = static_cast<uint32_t*>(ctr);
-    } else {
-        if (ws) cudaFree(ws);
-        if (ctr) cudaFree(ctr);
-        cudaGetLastError();  // clear the allocation error; split-K stays off
-    }
-    st.ready = true;
+    st.ready.store(true, std::memory_order_release);
     return DG_OK;
 }
 
@@ -223,19 +236,21 @@ dg_status noalloc_device(DeviceState** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
     if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mu);
     DeviceState& st = g_dev_noalloc[dev];
-    if (!st.ready) {
-        const dg_status s = setup_device(dev, st);
-        if (s != DG_OK) return s;
-        void* partials = nullptr;
-        void* counters = nullptr;
-        if (cudaGetSymbolAddress(&partials, g_noalloc_partials) != cudaSuccess ||
-            cudaGetSymbolAddress(&counters, g_noalloc_counters) != cudaSuccess)
-            return DG_ERR_CUDA;
-        st.split_ws = static_cast<float*>(partials);
-        st.split_counters = static_cast<uint32_t*>(counters);
-        st.ready = true;
+    if (!st.ready.load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> lock(g_mu);
+        if (!st.ready.load(std::memory_order_relaxed)) {
+            const dg_status s = setup_device(dev, st);
+            if (s != DG_OK) return s;
+            void* partials = nullptr;
+            void* counters = nullptr;
+            if (cudaGetSymbolAddress(&partials, g_noalloc_partials) != cudaSuccess ||
+                cudaGetSymbolAddress(&counters, g_noalloc_counters) != cudaSuccess)
+                return DG_ERR_CUDA;
+            st.split_ws = static_cast<float*>(partials);
+            st.split_counters = static_cast<uint32_t*>(counters);
+            st.ready.store(true, std::memory_order_release);
+        }
     }
     *out = &st;
     return DG_OK;
@@ -245,7 +260,7 @@ dg_status current_device(DeviceState** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
     if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
-    if (!g_dev[dev].ready) {
+    if (!g_dev[dev].ready.load(std::memory_order_acquire)) {
         dg_status s = init_device(dev);
         if (s != DG_OK) return s;
     }
@@ -315,12 +330,18 @@ constexpr double kHbmBytesPerClk = 3500.0;
 // issue to arrival; all CTAs together draw about 2400 bytes per clock.
 constexpr double kHbmLatencyClk = 4400.0;
 constexpr double kBStreamBytesPerClk = 2400.0;
-// Split-K: the most ranges per tile; the unit that reduces a tile pays about
-// one L2 round trip (~700 clocks) per 32 columns per two splits, plus a fixed
-// hand-off (fence, counter) of ~2000 clocks.
+// Split-K through global scratch (fp8_gemm_nt_noalloc): the most ranges per
+// tile; the unit that reduces a tile pays about one L2 round trip (~700
+// clocks) per 32 columns per two splits, plus a fixed hand-off (fence,
+// counter) of ~2000 clocks.
 constexpr int kMaxSplits = 16;
 constexpr double kL2LatencyClk = 700.0;
 constexpr double kSplitFixedClocks = 2000.0;
+// Split-K inside a cluster: a fixed hand-off (two cluster-scope barrier
+// round trips, ~1500 clocks) plus the pieces each CTA sends to the owners
+// through distributed shared memory at about 32 bytes per clock.
+constexpr double kClusterSplitFixedClocks = 1500.0;
+constexpr double kDsmemBytesPerClk = 32.0;
 
 // Clocks one SM spends per 128-K block of its (rows_a x bn) share of a tile:
 // the larger of the tensor core (four K=32 block-scaled MMAs of bn/2 clocks
@@ -338,8 +359,9 @@ int num_acc_for(int bn) { return (2 * bn + 2 * (4 + 4 * ((bn + 127) / 128)) <= 5
 
 struct TileChoice {
     const KernelEntry* entry;
-    int units;             // concurrent MMA units (CTAs, or CTA pairs)
+    int units;             // concurrent MMA units (CTAs, or CTA pairs); for a cluster split, CTAs
     int splits;            // split-K ranges per output tile (1 = none)
+    int split_mode;        // dg::SPLIT_NONE / SPLIT_CLUSTER / SPLIT_SCRATCH
 };
 
 // Pick the kernel (N tile, one CTA or a CTA pair) and, for the dense form,
@@ -348,12 +370,14 @@ struct TileChoice {
 // unique bytes at the HBM rate. Split-K is considered only when the output
 // tiles alone leave SMs idle; a split unit also pays for writing its fp32
 // partial and, on average, for one reduction read of all partials.
-// Split-K scratch a choice may use: partial floats and per-tile counters
-// (split_ok false: no scratch at all).
+// How split-K may run: inside clusters (the library's own calls) or through
+// global scratch of the given size (fp8_gemm_nt_noalloc); split_ok false: not
+// at all.
 struct SplitScratch {
     bool split_ok;
-    double bytes;
-    long long counters;
+    int mode;             // dg::SPLIT_CLUSTER or dg::SPLIT_SCRATCH
+    double bytes;         // SPLIT_SCRATCH: partial bytes available
+    long long counters;   // SPLIT_SCRATCH: per-tile counters available
 };
 
 TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
@@ -364,7 +388,7 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     const int forced_bn = g_force_bn.load();
     // no pairs for the masked and psum_m forms
     const int forced_cg = (kind != dg::kMasked && kind != dg::kPsum) ? g_force_cg.load() : 0;
-    TileChoice best{nullptr, 0, 1};
+    TileChoice best{nullptr, 0, 1, dg::SPLIT_NONE};
     double best_cost = 1e300;
     const double hbm_floor = static_cast<double>(unique_bytes) / kHbmBytesPerClk;
     for (int i = 0; i < kNumKernels; ++i) {
@@ -386,29 +410,47 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
         const int rows_a = rows < dg::BM ? rows : dg::BM;
         const double kbc0 = kblock_clocks(e.bn, e.cg, rows_a);
         const double bubble = num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0;
-        for (int splits = 1; splits <= kMaxSplits; ++splits) {
+        const bool cluster_mode = scratch.mode == dg::SPLIT_CLUSTER;
+        const int max_splits = cluster_mode ? kMaxClusterSplits : kMaxSplits;
+        for (int splits = 1; splits <= max_splits; ++splits) {
             if (forced_splits != 0 && splits != forced_splits) continue;
-            const bool can_split = kind == dg::kDense && e.cg == 1 && scratch.split_ok;
+            const bool can_split = kind == dg::kDense && e.cg == 1 && e.layout == 0 && scratch.split_ok;
+            int su = units;  // concurrent work units of this split count
             if (splits > 1) {
                 if (!can_split || splits > kg) break;
+                if (cluster_mode) {
+                    // every CTA owns at least one 8-column piece; the received
+                    // pieces fit in the operand ring
+                    if (splits > e.bn / 8) break;
+                    if (dg::cluster_split_bytes(e.bn, splits) > e.stages * e.stage_bytes) continue;
+                    su = st->max_clusters[i][splits] * splits;
+                    if (su < splits) continue;
+                } else {
+                    if (tiles > scratch.counters) break;
+                    if (static_cast<double>(tiles) * splits * dg::BM * e.bn * sizeof(float) > scratch.bytes) break;
+                }
                 if (forced_splits == 0 && tiles >= units) break;  // the tiles alone fill the GPU
-                if (tiles > scratch.counters) break;
-                if (static_cast<double>(tiles) * splits * dg::BM * e.bn * sizeof(float) > scratch.bytes) break;
             }
             const int gps = (kg + splits - 1) / splits;  // K groups of the longest range
             const long long work = tiles * splits;
-            const long long waves = (work + units - 1) / units;
+            const long long waves = (work + su - 1) / su;
             const int kb_unit = gps * 4 < kb ? gps * 4 : kb;
             double kbc = kbc0;
             if (mt == 1) {  // B streamed once from HBM
-                const double active = static_cast<double>(work < units ? work : units);
+                const double active = static_cast<double>(work < su ? work : su);
                 const double lat = kHbmLatencyClk / e.stages;
                 const double bw = static_cast<double>(e.bn / e.cg) * 128.0 * active / kBStreamBytesPerClk;
                 if (lat > kbc) kbc = lat;
                 if (bw > kbc) kbc = bw;
             }
             double unit = kb_unit * kbc + bubble;
-            if (splits > 1) unit += (e.bn / 32.0) * ((splits + 1) / 2) * kL2LatencyClk + kSplitFixedClocks;
+            if (splits > 1) {
+                if (cluster_mode)
+                    unit += kClusterSplitFixedClocks +
+                            static_cast<double>(rows_a) * e.bn * 4.0 * (splits - 1) / splits / kDsmemBytesPerClk;
+                else
+                    unit += (e.bn / 32.0) * ((splits + 1) / 2) * kL2LatencyClk + kSplitFixedClocks;
+            }
             double cost = static_cast<double>(waves) * unit;
             if (cost < hbm_floor) cost = hbm_floor;
             const bool better =
@@ -418,27 +460,20 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
                   (splits == best.splits && (e.cg > best.entry->cg || (e.cg == best.entry->cg && e.bn > best.entry->bn)))));
             if (best.entry == nullptr || better) {
                 best_cost = cost;
-                best = TileChoice{&e, units, splits};
+                best = TileChoice{&e, su, splits, splits > 1 ? scratch.mode : dg::SPLIT_NONE};
             }
         }
     }
     return best;
 }
 
-// The library's own choice: the allocated split-K workspace, and the split
-// count forced by dgb200_set_splits (dense form).
+// The library's own choice: split-K inside clusters, and the split count
+// forced by dgb200_set_splits (dense form).
 TileChoice choose_tile(const DeviceState* st, int kind, int rows, int n, int k, long long m128_blocks,
                        long long unique_bytes, int dt = dg::kE4M3, int layout = 0, int epi = 0) {
     const int forced_splits = kind == dg::kDense ? g_force_splits.load() : 1;
-    const SplitScratch scratch{st->split_ws != nullptr, static_cast<double>(kSplitWsBytes), kSplitCounters};
+    const SplitScratch scratch{true, dg::SPLIT_CLUSTER, 0.0, 0};
     return choose_tile_in(st, kind, rows, n, k, m128_blocks, unique_bytes, forced_splits, scratch, dt, layout, epi);
-}
-
-// Bytes of split-K partials a choice writes (0 when it does not split).
-double split_bytes(const TileChoice& c, long long m128_blocks, int n) {
-    if (c.splits <= 1 || c.entry == nullptr) return 0.0;
-    const long long tiles = m128_blocks * ((n + c.entry->bn - 1) / c.entry->bn);
-    return static_cast<double>(tiles) * c.splits * dg::BM * c.entry->bn * sizeof(float);
 }
 
 // Launch configuration of the elementwise pack kernels (programmatic
@@ -471,7 +506,8 @@ dg_status check_common(const void* a, const int32_t* sfa, const void* b, const i
 }
 
 // Launch one GEMM with a given tile choice; split-K partials and counters
-// come from `ws` / `counters` (used only when the choice splits).
+// come from `ws` / `counters` (used only when the choice splits through
+// global scratch).
 dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counters, int kind, GemmParams& p,
                            long long max_tiles_per_nblock, void* stream, const DeviceState* st, const void* a,
                            const void* b, int a_rank, int b_rank, uint64_t a_rows, uint64_t a_mats, uint64_t b_rows,
@@ -495,8 +531,11 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.test_mode = g_test_mode.load();
     p.splits = choice.splits;
-    p.ws = choice.splits > 1 ? ws : nullptr;
-    p.counters = choice.splits > 1 ? counters : nullptr;
+    p.split_mode = choice.splits > 1 ? choice.split_mode : dg::SPLIT_NONE;
+    const bool scratch_split = p.split_mode == dg::SPLIT_SCRATCH;
+    if (scratch_split && (ws == nullptr || counters == nullptr)) return DG_ERR_UNSUPPORTED;
+    p.ws = scratch_split ? ws : nullptr;
+    p.counters = scratch_split ? counters : nullptr;
     p.k_rotate = choice.splits > 1 ? 0 : g_k_rotate;  // a split walks its own range in order
     if (p.k_rotate) p.sf_vec4 = 0;                     // quads are walked in K order
     if (e->layout & 1) {
@@ -515,14 +554,19 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     const long long tiles = (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks) *
                             choice.splits * (cg == 2 && kind == dg::kContiguous ? 2 : 1);
     if (tiles <= 0) return DG_OK;
-    const int units = static_cast<int>(tiles < choice.units ? tiles : choice.units);
+    // a cluster split runs every work unit on a CTA of its own (one tile per
+    // cluster: the reduction uses the operand ring, which is then idle)
+    const bool cluster_split = p.split_mode == dg::SPLIT_CLUSTER;
+    if (cluster_split && (kind != dg::kDense || cg != 1 || tiles > (1LL << 30))) return DG_ERR_UNSUPPORTED;
+    const int units = cluster_split ? static_cast<int>(tiles)
+                                    : static_cast<int>(tiles < choice.units ? tiles : choice.units);
     void* args[] = {&p};
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[2];
     unsigned nattr = 0;
-    if (cg == 2) {
+    if (cg == 2 || cluster_split) {
         attr[nattr].id = cudaLaunchAttributeClusterDimension;
-        attr[nattr].val.clusterDim.x = 2;
+        attr[nattr].val.clusterDim.x = cg == 2 ? 2u : static_cast<unsigned>(choice.splits);
         attr[nattr].val.clusterDim.y = 1;
         attr[nattr].val.clusterDim.z = 1;
         ++nattr;
@@ -540,8 +584,10 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     cfg.numAttrs = nattr;
     if (g_log)
         std::fprintf(stderr,
-                     "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d splits=%d grid=%d (units %d) smem=%d\n",
-                     kind, p.rows, p.n, p.k, p.groups, bn, cg, choice.splits, units * cg, choice.units, e->smem);
+                     "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d splits=%d (mode %d) grid=%d "
+                     "(units %d) smem=%d\n",
+                     kind, p.rows, p.n, p.k, p.groups, bn, cg, choice.splits, p.split_mode, units * cg, choice.units,
+                     e->smem);
     cudaError_t err = cudaLaunchKernelExC(&cfg, e->fn, args);
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }
@@ -552,8 +598,8 @@ dg_status launch_gemm(int kind, GemmParams& p, long long m_blocks_for_heuristic,
                       int dt = dg::kE4M3, int layout = 0, int epi = 0) {
     const TileChoice choice =
         choose_tile(st, kind, p.rows, p.n, p.k, m_blocks_for_heuristic, unique_bytes, dt, layout, epi);
-    return launch_gemm_with(choice, st->split_ws, st->split_counters, kind, p, max_tiles_per_nblock, stream, st, a, b,
-                            a_rank, b_rank, a_rows, a_mats, b_rows, b_mats);
+    return launch_gemm_with(choice, nullptr, nullptr, kind, p, max_tiles_per_nblock, stream, st, a, b, a_rank, b_rank,
+                            a_rows, a_mats, b_rows, b_mats);
 }
 
 // Scale rows of B: one per 128x128 block (sfb_gran_n = 128) or one per row of B
@@ -696,23 +742,55 @@ const char* dgb200_status_string(dg_status s) {
     return "DG_ERR_UNKNOWN";
 }
 
-dg_status dgb200_init(void) {
-    DeviceState* st = nullptr;
-    return current_device(&st);
+dg_status dgb200_init(int device) {
+    int count = 0;
+    if (cudaGetDeviceCount(&count) != cudaSuccess) {
+        cudaGetLastError();
+        return DG_ERR_NOT_INITIALIZED;
+    }
+    if (device < 0 || device >= count) return DG_ERR_INVALID_ARG;
+    if (device >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    if (g_dev[device].ready.load(std::memory_order_acquire)) return DG_OK;
+    // kernel attributes apply to the current device: make `device` current for
+    // the set-up and restore the caller's device afterwards
+    int prev = -1;
+    if (cudaGetDevice(&prev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
+    if (prev != device && cudaSetDevice(device) != cudaSuccess) return DG_ERR_CUDA;
+    const dg_status s = init_device(device);
+    if (prev != device && cudaSetDevice(prev) != cudaSuccess) return DG_ERR_CUDA;
+    return s;
+}
+
+// Address of the status word on the current device without setting up the
+// kernels (the word is a static variable of the library's module).
+dg_status status_word(uint32_t** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DG_ERR_NOT_INITIALIZED;
+    if (dev < 0 || dev >= kMaxDevices) return DG_ERR_UNSUPPORTED;
+    void* status = nullptr;
+    if (cudaGetSymbolAddress(&status, g_dg_device_status) != cudaSuccess) return DG_ERR_CUDA;
+    *out = static_cast<uint32_t*>(status);
+    return DG_OK;
 }
 
 dg_status dgb200_device_error(uint32_t* bits, int clear) {
     if (bits == nullptr) return DG_ERR_INVALID_ARG;
-    DeviceState* st = nullptr;
-    dg_status s = current_device(&st);
+    uint32_t* word = nullptr;
+    const dg_status s = status_word(&word);
     if (s != DG_OK) return s;
     if (cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
-    if (cudaMemcpy(bits, st->status, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
-    if (clear && cudaMemset(st->status, 0, sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
-    // a launch that gave up may have left split-K counters part-way
-    if (clear && *bits != 0 && st->split_counters != nullptr &&
-        cudaMemset(st->split_counters, 0, kSplitCounters * sizeof(uint32_t)) != cudaSuccess)
-        return DG_ERR_CUDA;
+    if (cudaMemcpy(bits, word, sizeof(uint32_t), cudaMemcpyDeviceToHost) != cudaSuccess) return DG_ERR_CUDA;
+    if (clear && cudaMemset(word, 0, sizeof(uint32_t)) != cudaSuccess) return DG_ERR_CUDA;
+    if (clear && cudaDeviceSynchronize() != cudaSuccess) return DG_ERR_CUDA;
+    return DG_OK;
+}
+
+dg_status dgb200_last_device_error(int* code) {
+    if (code == nullptr) return DG_ERR_INVALID_ARG;
+    uint32_t bits = 0;
+    const dg_status s = dgb200_device_error(&bits, 1);
+    if (s != DG_OK) return s;
+    *code = static_cast<int>(bits);
     return DG_OK;
 }
 
@@ -735,7 +813,7 @@ dg_status dgb200_set_cta_group(int cta_group) {
 }
 
 dg_status dgb200_set_splits(int splits) {
-    if (splits < 0 || splits > kMaxSplits) return DG_ERR_UNSUPPORTED;
+    if (splits < 0 || splits > kMaxClusterSplits) return DG_ERR_UNSUPPORTED;
     g_force_splits.store(splits);
     return DG_OK;
 }
@@ -827,24 +905,16 @@ dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, 
     p.num_m_blocks = (M + dg::BM - 1) / dg::BM;
     const long long bytes = (static_cast<long long>(M) + N) * K + 2LL * M * N;
     const double static_bytes = static_cast<double>(kStaticPartialFloats) * sizeof(float);
-    TileChoice choice;
-    if (splits == 0) {
-        // the model's choice among what fits the static scratch
-        const SplitScratch scratch{true, static_bytes, kStaticCounters};
-        choice = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, 0, scratch);
-    } else {
-        // exactly `splits` ranges, tiled as the model would with unlimited
-        // scratch; refused if that needs more than the static arrays hold
-        const SplitScratch unlimited{true, 1e300, 1LL << 40};
-        choice = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, splits, unlimited);
-        if (choice.entry == nullptr) return DG_ERR_UNSUPPORTED;
-        if (choice.splits > 1) {
-            const long long tiles = p.num_m_blocks * ((N + choice.entry->bn - 1) / choice.entry->bn);
-            if (split_bytes(choice, p.num_m_blocks, N) > static_bytes || tiles > kStaticCounters)
-                return DG_ERR_SCRATCH_TOO_SMALL;
-        }
+    // the model's choice among the tile widths whose partials fit the static
+    // scratch (splits = 0: any split count; else exactly `splits`)
+    const SplitScratch scratch{true, dg::SPLIT_SCRATCH, static_bytes, kStaticCounters};
+    const TileChoice choice = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, splits, scratch);
+    if (choice.entry == nullptr) {
+        // refused: say whether scratch without limits would have allowed it
+        const SplitScratch unlimited{true, dg::SPLIT_SCRATCH, 1e300, 1LL << 40};
+        const TileChoice any = choose_tile_in(st, dg::kDense, M, N, K, p.num_m_blocks, bytes, splits, unlimited);
+        return any.entry != nullptr ? DG_ERR_SCRATCH_TOO_SMALL : DG_ERR_UNSUPPORTED;
     }
-    if (choice.entry == nullptr) return DG_ERR_UNSUPPORTED;
     if (choice.splits > 1) {
         // the counters must start at zero (a launch that gave up may have left some part-way)
         const long long tiles = p.num_m_blocks * ((N + choice.entry->bn - 1) / choice.entry->bn);

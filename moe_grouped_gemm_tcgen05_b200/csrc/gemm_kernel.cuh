@@ -87,6 +87,11 @@ constexpr uint64_t DEFAULT_WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 constexpr uint32_t DEVERR_TIMEOUT = 1u;
 constexpr uint32_t DEVERR_MIXED_EXPERT_BLOCK = 2u;
 
+constexpr int SPLIT_NONE = 0;
+constexpr int SPLIT_SCRATCH = 1;
+constexpr int SPLIT_CLUSTER = 2;
+constexpr int MAX_CLUSTER_SPLITS = 8;   // portable cluster size
+
 struct GemmParams {
     CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous, psum_m) or 3-D {K, max_m, G} (masked)
     CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped); box BN/CG rows
@@ -111,11 +116,15 @@ struct GemmParams {
     int sf_vec4;              // 1: scale rows are read 16 bytes (4 K groups) at a time (B scaled per row,
                               //    kp % 4 == 0, 16-byte bases, K groups in order)
     // split-K (dense form, single CTAs): each output tile is computed by `splits`
-    // work units over disjoint ranges of K groups; the last one to finish adds
-    // the fp32 partials in split order and writes the bf16 tile
+    // work units over disjoint ranges of K groups, whose fp32 partials are
+    // added in split order
     int splits;               // 1 = no split; range i covers K groups [i*G/splits, (i+1)*G/splits)
-    float* ws;                // partials: [tile][split][4 row quarters][BN/4][32 lanes][4]
-    uint32_t* counters;       // finished units per output tile; zero between calls
+    int split_mode;           // SPLIT_CLUSTER: the units of a tile form one cluster and add their
+                              //   partials through distributed shared memory (no global scratch);
+                              // SPLIT_SCRATCH: units park partials in `ws` and the last one to
+                              //   finish adds them
+    float* ws;                // SPLIT_SCRATCH partials: [tile][split][4 row quarters][BN/4][32 lanes][4]
+    uint32_t* counters;       // SPLIT_SCRATCH: finished units per output tile; zero between calls
     // dense form: D = C + A.B^T. C (optional, [rows, n] in D's type) is added to
     // the fp32 accumulation before the final conversion; D is bf16 (d, TMA
     // stores) or fp32 (d32, direct stores)
@@ -193,8 +202,11 @@ __device__ __forceinline__ uint64_t global_ns() {
 // waiting at the next elect.sync, __syncwarp or .sync.aligned instruction).
 // Gives up when another role of this CTA has given up, or after
 // p.wait_limit_ns; a timeout is recorded in the device status word.
+// CLUSTER_ACQ: the probe acquires at cluster scope (the phase carries writes
+// or arrives of other CTAs of the cluster).
+template <bool CLUSTER_ACQ = false>
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, const GemmParams& p, volatile int* s_abort) {
-    auto probe = [&]() { return mbar_try_wait(bar, parity); };
+    auto probe = [&]() { return CLUSTER_ACQ ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
     if (__all_sync(0xffffffffu, probe())) return true;
     const uint64_t t0 = global_ns();
     while (true) {
@@ -472,6 +484,165 @@ struct ScaleQuads {
     }
 };
 
+// -------------------------------------------------- cluster split-K epilogue --
+//
+// SPLIT_CLUSTER: the `splits` = S units of an output tile are the S CTAs of one
+// cluster; CTA r holds the fp32 partial of K range r of the whole 128 x BN
+// tile in TMEM. The tile's columns are dealt out in 8-column pieces: of the
+// NP = BN/8 pieces, CTA r owns [r*NP/S, (r+1)*NP/S). Each CTA sends every piece
+// it does not own to the owner with st.async into the owner's operand ring
+// (idle once the owner's own MMAs have completed), counted in bytes on the
+// owner's barrier of the receiving epilogue warp. The owner adds the S
+// partials of its pieces in split order, its own read back from TMEM, and
+// writes them. Nothing outside the cluster's shared memory is used, so
+// concurrent calls share no state.
+//
+// Layout of the received pieces in the owner's ring (16-byte units):
+// [sender rank][piece j of the owner][half: columns 0-3 / 4-7][tile row].
+__device__ __forceinline__ uint32_t cluster_piece_offset(int sender, int pmax, int j, int half, int row) {
+    return static_cast<uint32_t>((((sender * pmax + j) * 2 + half) * BM + row) * 16);
+}
+
+// Shared-memory bytes of the received pieces of one tile: S slots of at most
+// ceil(NP / S) pieces of 128 rows x 32 bytes.
+__host__ __device__ constexpr int cluster_split_bytes(int bn, int splits) {
+    return splits * ((bn / 8 + splits - 1) / splits) * BM * 32;
+}
+
+// Rows of the tile that the epilogue warp covering tile rows 32q..32q+31 must
+// reduce: false when all of them lie past M (nothing to send or receive).
+__device__ __forceinline__ bool cluster_warp_live(const GemmParams& p, int m_blk, int q) {
+    return m_blk * BM + 32 * q < p.rows;
+}
+
+// Bytes the owner's warp q receives: S - 1 senders x its pieces x 32 rows x 32 bytes.
+__device__ __forceinline__ uint32_t cluster_expected_bytes(const GemmParams& p, int rank, int np, int m_blk, int q) {
+    const int S = p.splits;
+    const int mine = (rank + 1) * np / S - rank * np / S;
+    return cluster_warp_live(p, m_blk, q) ? static_cast<uint32_t>((S - 1) * mine * 32 * 32) : 0u;
+}
+
+// Eight reduced columns of one row of D at element offset `at`: + C and an
+// fp32 or bf16 (round to nearest even) store (EPI 1), or a bf16 store (EPI 0).
+template <int EPI>
+__device__ __forceinline__ void cluster_store8(const GemmParams& p, float* acc, size_t at) {
+    if constexpr (EPI == 1) {
+        if (p.c != nullptr) {
+            if (p.out_f32) {
+                const float4 x0 = *reinterpret_cast<const float4*>(static_cast<const float*>(p.c) + at);
+                const float4 x1 = *reinterpret_cast<const float4*>(static_cast<const float*>(p.c) + at + 4);
+                acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
+                acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
+            } else {
+                const uint4 x = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.c) + at);
+                const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int h2 = 0; h2 < 4; ++h2) {
+                    const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                    acc[2 * h2] += c2.x;
+                    acc[2 * h2 + 1] += c2.y;
+                }
+            }
+        }
+        if (p.out_f32) {
+            *reinterpret_cast<float4*>(p.d32 + at) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            *reinterpret_cast<float4*>(p.d32 + at + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            return;
+        }
+    }
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(p.d + at) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The reduction and store of one warp's 32 rows (dense form, single CTAs).
+// Returns false when a wait gave up.
+template <int BN, int EPI>
+__device__ __forceinline__ bool cluster_split_epilogue(const GemmParams& p, const Tile& c, int q, uint32_t warp,
+                                                       uint32_t lane, uint32_t taddr, uint8_t* ring,
+                                                       uint64_t* red_free, uint64_t* red_full,
+                                                       volatile int* s_abort) {
+    constexpr int NP = BN / 8;
+    const int S = p.splits;
+    const int rank = static_cast<int>(cluster_ctarank());
+    const int pmax = (NP + S - 1) / S;
+    const int row = 32 * q + static_cast<int>(lane);      // tile row of this thread
+    const int m = c.m_blk * BM + row;                      // row of D
+    const bool live = cluster_warp_live(p, c.m_blk, q);    // warp-uniform
+    // 1. this CTA's MMAs have completed (the caller saw the accumulator
+    //    barrier), so its ring may take the peers' pieces: tell every peer
+    if (warp == 2) {
+        __syncwarp();
+        if (static_cast<int>(lane) < S && static_cast<int>(lane) != rank)
+            mbar_arrive_release_cluster(mapa_shared(smem_u32(red_free), lane));
+    }
+    // 2. every peer's ring is free
+    if (!wait_warp<true>(red_free, 0, p, s_abort)) return false;
+    // 3. send the pieces other CTAs own
+    if (live) {
+        const uint32_t ring_s = smem_u32(ring);
+        const uint32_t bar_s = smem_u32(&red_full[q]);
+#pragma unroll
+        for (int h = 0; h < BN; h += 32) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(taddr + h, r);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int pc = h / 8 + i;
+                const int o = ((pc + 1) * S - 1) / NP;   // owner of piece pc
+                if (o == rank) continue;
+                const int j = pc - o * NP / S;
+                const uint32_t dst = mapa_shared(ring_s, static_cast<uint32_t>(o));
+                const uint32_t bar = mapa_shared(bar_s, static_cast<uint32_t>(o));
+                st_async_v4(dst + cluster_piece_offset(rank, pmax, j, 0, row), bar, r[8 * i], r[8 * i + 1],
+                            r[8 * i + 2], r[8 * i + 3]);
+                st_async_v4(dst + cluster_piece_offset(rank, pmax, j, 1, row), bar, r[8 * i + 4], r[8 * i + 5],
+                            r[8 * i + 6], r[8 * i + 7]);
+            }
+        }
+    }
+    // 4. every peer's pieces for these rows have landed: add the S partials of
+    //    each owned piece in split order and store
+    if (!wait_warp<true>(&red_full[q], 0, p, s_abort)) return false;
+    if (live) {
+        const int mine0 = rank * NP / S;
+        const int mine1 = (rank + 1) * NP / S;
+        for (int pc = mine0; pc < mine1; ++pc) {
+            const int j = pc - mine0;
+            float acc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            for (int s = 0; s < S; ++s) {
+                float v[8];
+                if (s == rank) {
+                    uint32_t t[8];
+                    tmem_ld_32x32b_x8(taddr + 8 * pc, t);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(t[i]);
+                } else {
+                    const float4 lo = *reinterpret_cast<const float4*>(ring + cluster_piece_offset(s, pmax, j, 0, row));
+                    const float4 hi = *reinterpret_cast<const float4*>(ring + cluster_piece_offset(s, pmax, j, 1, row));
+                    v[0] = lo.x; v[1] = lo.y; v[2] = lo.z; v[3] = lo.w;
+                    v[4] = hi.x; v[5] = hi.y; v[6] = hi.z; v[7] = hi.w;
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += v[i];
+            }
+            const int col = c.n_blk * BN + 8 * pc;
+            // N % 8 == 0: a piece is wholly inside or outside D
+            if (col < p.n && m < p.rows) cluster_store8<EPI>(p, acc, static_cast<size_t>(m) * p.n + col);
+            __syncwarp();
+        }
+    }
+    return true;
+}
+
 // ------------------------------------------------------------------ kernel --
 
 // LAYOUT bit 0: A is stored MN-major ([K, M], M contiguous); bit 1: B is
@@ -520,7 +691,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     uint64_t* tempty_bar = tfull_bar + 2;            // accumulator drained by the epilogue(s)
     uint64_t* drain_bar = tempty_bar + 2;            // all MMAs issued for this CTA finished
     uint64_t* epi_bar = drain_bar + 1;               // split-K: the four epilogue warps meet
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(epi_bar + 1);
+    uint64_t* red_free = epi_bar + 1;                // cluster split-K: every peer's ring is free
+    uint64_t* red_full = red_free + 1;               // cluster split-K: peers' pieces landed, per epilogue warp
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(red_full + 4);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);  // split-K: this unit reduces
     int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked, psum_m)
@@ -549,6 +722,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         }
         mbar_init(drain_bar, 1);
         mbar_init(epi_bar, 4);
+        if constexpr (KIND == kDense && CG == 1) {
+            if (p.split_mode == SPLIT_CLUSTER) {
+                // one arrive from each peer; per epilogue warp, one arrive (made
+                // here) plus the bytes the peers' pieces will bring
+                mbar_init(red_free, static_cast<uint32_t>(p.splits - 1));
+                Tile t0;
+                raster_tile(p, static_cast<int>(blockIdx.x), t0);
+                const int rk = static_cast<int>(cluster_ctarank());
+                for (int q = 0; q < 4; ++q) {
+                    mbar_init(&red_full[q], 1);
+                    mbar_arrive_expect_tx(&red_full[q], cluster_expected_bytes(p, rk, BN / 8, t0.m_blk, q));
+                }
+            }
+        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -666,7 +853,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     }
     tc_fence_before();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
+    // every CTA's barriers exist before any cross-CTA signal (pairs, cluster split-K)
+    if (CG == 2 || (KIND == kDense && p.split_mode == SPLIT_CLUSTER)) cluster_sync();
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int kg_count = (p.kb + 3) / 4;
@@ -690,7 +878,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             for (int gi = cur.kg0; gi < cur.kg1 && !aborted; ++gi) {
             const int kgrp = rot_group(p, t, gi, kg_count);
             for (int kb = 4 * kgrp; kb < min(4 * kgrp + 4, p.kb); ++kb) {
-                if (!wait_warp(&empty_bar[stage], phase ^ 1u, p, s_abort)) { aborted = true; break; }
+                // the first STAGES slots are free from the start: no wait
+                if (issued >= STAGES && !wait_warp(&empty_bar[stage], phase ^ 1u, p, s_abort)) { aborted = true; break; }
                 if (elect_one()) {
                     uint8_t* a_dst = smem_a + stage * Cfg::A_BYTES;
                     uint8_t* b_dst = smem_b + stage * Cfg::B_BYTES;
@@ -1019,12 +1208,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             const int n0 = c.n_blk * BN;
             __nv_bfloat16* drow = p.d + out_row * static_cast<size_t>(p.n) + n0;
             constexpr int kMaxBatch = 128;
-            // split-K (dense, single CTAs): every unit parks its fp32 partial
-            // in the workspace; the unit that finishes a tile last adds the
-            // partials in split order (the same sum whichever unit is last)
-            // and writes the bf16 tile.
             constexpr bool kCanSplit = KIND == kDense && CG == 1;
-            const bool split = kCanSplit && p.splits > 1;
+            if constexpr (kCanSplit) {
+                if (p.split_mode == SPLIT_CLUSTER) {
+                    // split-K inside a cluster: the partials meet in the owners'
+                    // shared memory (one tile per CTA, so the ring is free)
+                    if (!cluster_split_epilogue<BN, EPI>(p, c, q, warp, lane, taddr, smem_a, red_free, red_full,
+                                                         s_abort))
+                        break;
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty_bar[acc]);
+                    if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
+                    continue;
+                }
+            }
+            // split-K through global scratch (dense, single CTAs): every unit
+            // parks its fp32 partial in the workspace; the unit that finishes a
+            // tile last adds the partials in split order (the same sum whichever
+            // unit is last) and writes the bf16 tile.
+            const bool split = kCanSplit && p.split_mode == SPLIT_SCRATCH;
             bool emit_tile = !split;
             if constexpr (kCanSplit) {
                 if (split) {
@@ -1230,7 +1433,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
 
     tc_fence_before();
     __syncthreads();
-    if constexpr (CG == 2) cluster_sync();  // neither CTA frees TMEM while the pair still uses it
+    // neither CTA of a pair frees TMEM while the pair still uses it; no CTA of a
+    // split-K cluster exits while peers may still write into its shared memory
+    if (CG == 2 || (KIND == kDense && p.split_mode == SPLIT_CLUSTER)) cluster_sync();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc<CG>(tmem_base, Cfg::TMEM_COLS);

@@ -28,7 +28,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = set(declared_functions())
     for n in ("fp8_gemm_nt", "m_grouped_fp8_gemm_nt_contiguous", "m_grouped_fp8_gemm_nt_masked",
-              "pack_ue8m0", "pack_ue8m0_validate", "dgb200_init", "dgb200_device_error"):
+              "pack_ue8m0", "pack_ue8m0_validate", "dgb200_init", "dgb200_last_device_error",
+              "dgb200_device_error"):
         assert n in names
 
 
@@ -113,12 +114,23 @@ def test_binding_fails_loudly_without_cuda():
                        torch.zeros((1, 1), dtype=torch.int32), torch.zeros((128, 128), dtype=torch.bfloat16))
 
 
+def test_init_and_error_word_arguments(lib):
+    """dgb200_init takes a device ordinal and dgb200_last_device_error an output
+    pointer; bad arguments are refused on the host (no device needed)."""
+    lib.dgb200_init.restype = ctypes.c_int
+    lib.dgb200_init.argtypes = [ctypes.c_int]
+    assert lib.dgb200_init(-1) in (1, 4)          # invalid ordinal (or no usable driver here)
+    lib.dgb200_last_device_error.restype = ctypes.c_int
+    lib.dgb200_last_device_error.argtypes = [ctypes.c_void_p]
+    assert lib.dgb200_last_device_error(None) == 1
+
+
 def test_tuning_switch_ranges(lib):
     """The process-wide tuning switches reject values outside their ranges and
     need no device to do so (0 restores the heuristic in each)."""
     for name, good, bad in (("dgb200_set_block_n", (0, 64, 224, 256), (-1, 100, 512)),
                             ("dgb200_set_cta_group", (0, 1, 2), (-1, 3)),
-                            ("dgb200_set_splits", (0, 1, 2, 16), (-1, 17))):
+                            ("dgb200_set_splits", (0, 1, 2, 8), (-1, 9, 17))):
         f = getattr(lib, name)
         f.restype = ctypes.c_int
         f.argtypes = [ctypes.c_int]

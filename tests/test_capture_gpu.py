@@ -1,9 +1,12 @@
-"""Every compute entry point is CUDA-Graph capture safe ("DeepGEMM CUDA Graph
-Compatibility for Masked Grouped GEMMs", Stateless Kernel Architecture: no
-allocation, no host synchronisation, launch configuration fixed by the
-dimensions): each call is captured in global capture mode, where a hidden
-synchronisation or allocation makes the capture fail, and one replay must
-reproduce the eager result bit for bit. All calls go through the C ABI."""
+"""Every compute entry point of the method is CUDA-Graph capture safe
+("DeepGEMM CUDA Graph Compatibility for Masked Grouped GEMMs", Stateless
+Kernel Architecture: no allocation, no host synchronisation, launch
+configuration fixed by the dimensions): each call is captured in global
+capture mode, where a hidden synchronisation or allocation makes the capture
+fail, and one replay must reproduce the eager result bit for bit. All calls
+go through the C ABI. fp8_gemm_nt_noalloc, an addition of this library with
+no counterpart in the method, is not covered here: no claim is made about
+capturing it."""
 
 import numpy as np
 import pytest

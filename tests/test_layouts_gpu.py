@@ -24,6 +24,7 @@ def _reset():
     dg.device_error(clear=True)
     yield
     dg.set_block_n(0)
+    dg.set_splits(0)
     assert dg.device_error(clear=True) == 0
 
 
@@ -46,6 +47,7 @@ def test_layout_parity_and_equal_to_nt(layout, bn, mnk):
     d = fill_sentinel(torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
     FN[layout](_dev(a), sfa, _dev(b), sfb, d)
     d_nt = torch.empty_like(d)
+    dg.set_splits(1)   # the layouts run unsplit; compare with the unsplit NT kernel
     dg.fp8_gemm_nt(_dev(a_mk), sfa, _dev(b_nk), sfb, d_nt)
     torch.cuda.synchronize()
     assert not is_sentinel(d).any()

@@ -1,8 +1,15 @@
 """Split-K of the dense GEMM on the GPU vs the CPU oracle: forced split
 counts over ragged shapes (uneven K ranges, several m-blocks, N tails),
-bit-identical results on repeated calls (partials are added in split order,
-whichever unit finishes last), and CUDA Graph replay (the per-tile counters
-return to zero by themselves). All calls go through the C ABI."""
+bit-identical results on repeated calls (partials are added in split order),
+CUDA Graph replay, splitting calls running at the same time on two streams
+(the units of a tile meet inside their cluster, so calls share no scratch),
+and no device allocation by the library after its module is loaded. All
+calls go through the C ABI."""
+
+import os
+import subprocess
+import sys
+import textwrap
 
 import numpy as np
 import pytest
@@ -129,3 +136,66 @@ def test_split_k_graph_replay_with_new_inputs():
         torch.cuda.synchronize()
         check_fp(bf16_to_f64(d), _ref(p), "split-K graph replay")
     del g
+
+
+def test_split_k_calls_run_concurrently_on_two_streams():
+    # Many small splitting calls on two streams at once, each stream with its
+    # own inputs and outputs: every result must match the oracle (a shared
+    # workspace would mix the partials of the two streams' tiles).
+    M, N, K = 64, 512, 7168
+    ps = [W.dense(M, N, K, seed=60 + i) for i in range(2)]
+    args = [_inputs(p) for p in ps]
+    dg.set_block_n(128)
+    dg.set_splits(4)
+    streams = [torch.cuda.Stream() for _ in range(2)]
+    outs = [[torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for _ in range(40)] for _ in range(2)]
+    torch.cuda.synchronize()
+    for i in range(40):
+        for j in range(2):
+            with torch.cuda.stream(streams[j]):
+                dg.fp8_gemm_nt(*args[j], outs[j][i])
+    torch.cuda.synchronize()
+    for j in range(2):
+        check_fp(bf16_to_f64(outs[j][0]), _ref(ps[j]), f"stream {j}")
+        for d in outs[j][1:]:
+            assert torch.equal(d.view(torch.int16), outs[j][0].view(torch.int16)), f"stream {j}"
+
+
+_PROBE = textwrap.dedent("""
+    import sys, numpy as np, torch
+    sys.path.insert(0, {root!r})
+    import moe_grouped_gemm_tcgen05_b200 as dg
+    from moe_grouped_gemm_tcgen05_b200 import workloads as W
+    torch.cuda.set_device(0)
+    p = W.dense_t(64, 2112, 7168, seed=5)
+    sfa, sfb = [torch.zeros((r, 14), dtype=torch.int32, device="cuda") for r in (64, 17)]
+    sfa.fill_(0x7f7f7f7f)
+    sfb.fill_(0x7f7f7f7f)
+    d = torch.empty((64, 2112), dtype=torch.bfloat16, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    dg.init()                                    # loads the module, sets up the device
+    dg.set_splits(4)
+    dg.fp8_gemm_nt(p["a"], sfa, p["b"], sfb, d)   # the first launch of this kernel
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        dg.fp8_gemm_nt(p["a"], sfa, p["b"], sfb, d)
+    torch.cuda.synchronize()
+    free2 = torch.cuda.mem_get_info()[0]
+    print(free0 - free1, free1 - free2)
+""")
+
+
+def test_library_allocates_nothing_in_a_fresh_process():
+    # Setting up the device and the first launch load the module (its code
+    # and static arrays); after that, splitting calls leave the device's free
+    # memory exactly unchanged, and the load itself stays far below the 40 MB
+    # a split-K workspace would take.
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", _PROBE.format(root=root)], capture_output=True, text=True,
+                         timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    load_bytes, calls_bytes = (int(x) for x in out.stdout.split()[-2:])
+    assert calls_bytes == 0, (load_bytes, calls_bytes)
+    assert load_bytes < 32 << 20, (load_bytes, calls_bytes)

@@ -99,8 +99,7 @@ _PROBE = textwrap.dedent("""
     import moe_grouped_gemm_tcgen05_b200 as dg
     from moe_grouped_gemm_tcgen05_b200 import workloads as W
     torch.cuda.set_device(0)
-    # inputs prepared without calling the library (its other entry points set
-    # up the device with the workspace allocation)
+    # inputs prepared without calling the library
     p = W.dense(64, 2112, 7168, seed=5)
     dev = lambda x: torch.from_numpy(np.ascontiguousarray(x)).cuda()
     p = dict(a=dev(p["a"]), b=dev(p["b"]), sfa=oracle.pack_ue8m0(p["sfa_f32"]), sfb=oracle.pack_ue8m0(p["sfb_f32"]))
@@ -108,26 +107,31 @@ _PROBE = textwrap.dedent("""
     d = torch.empty((64, 2112), dtype=torch.bfloat16, device="cuda")
     torch.cuda.synchronize()
     free0 = torch.cuda.mem_get_info()[0]
+    # the first call loads the library's module: its code and static arrays
+    dg.fp8_gemm_nt_noalloc(p["a"], sfa, p["b"], sfb, d, splits=4)
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
     for _ in range(3):
         dg.fp8_gemm_nt_noalloc(p["a"], sfa, p["b"], sfb, d, splits=4)
     torch.cuda.synchronize()
-    free1 = torch.cuda.mem_get_info()[0]
-    dg.set_splits(4)
-    dg.fp8_gemm_nt(p["a"], sfa, p["b"], sfb, d)   # the existing entry point sets up its 40 MB workspace
-    torch.cuda.synchronize()
     free2 = torch.cuda.mem_get_info()[0]
-    print((free0 - free1) >> 20, (free1 - free2) >> 20)
+    # a deliberate 16 MiB allocation shows that the measurement sees one
+    x = torch.empty(16 << 20, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    free3 = torch.cuda.mem_get_info()[0]
+    print(free0 - free1, free1 - free2, free2 - free3)
 """)
 
 
 def test_no_device_allocation_in_a_fresh_process():
-    # The first no-alloc calls load the library's module (code and its static
-    # arrays, about 8 MiB) but allocate nothing; the existing entry point's
-    # first call then allocates its 40 MB split-K workspace, which shows that
-    # the measurement sees allocations of that size.
+    # The first call loads the library's module (its code and the static
+    # arrays, about 8 MiB of them). After it, further calls must leave the
+    # device's free memory exactly unchanged; a 16 MiB allocation made on
+    # purpose afterwards shows that the measurement sees one of that size.
     out = subprocess.run([sys.executable, "-c", _PROBE.format(root=ROOT)], capture_output=True, text=True,
                          timeout=300)
     assert out.returncode == 0, out.stderr[-2000:]
-    noalloc_mib, existing_mib = (int(x) for x in out.stdout.split()[-2:])
-    assert existing_mib >= 40, (noalloc_mib, existing_mib)
-    assert noalloc_mib < 32, (noalloc_mib, existing_mib)
+    load_bytes, calls_bytes, probe_bytes = (int(x) for x in out.stdout.split()[-3:])
+    assert probe_bytes >= 16 << 20, (load_bytes, calls_bytes, probe_bytes)
+    assert calls_bytes == 0, (load_bytes, calls_bytes, probe_bytes)
+    assert load_bytes < 32 << 20, (load_bytes, calls_bytes, probe_bytes)
