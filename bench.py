@@ -244,6 +244,41 @@ def step_ops(dg, probs):
     return ops
 
 
+L2_BYTES = 126e6
+
+
+def steady_state_us(torch, dg, p, max_copies=32, replays=5):
+    """Per-call device time of one dense problem in a stream of back-to-back
+    calls: a graph of 2C calls cycling over C copies of the inputs (together at
+    least 4x L2, so no call finds its operands in L2), timed with events around
+    each replay; the median replay / 2C."""
+    M, N, K = p["M"], p["N"], p["K"]
+    C = int(min(max_copies, max(2, math.ceil(4 * L2_BYTES / dense_bytes(M, N, K)))))
+    sets = [(p["a"].clone(), p["sfa"].clone(), p["b"].clone(), p["sfb"].clone(), torch.empty_like(p["d"]))
+            for _ in range(C)]
+    calls = [lambda t=t: dg.fp8_gemm_nt(*t) for t in sets]
+    for f in calls:
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(2 * C):
+            calls[i % C]()
+    g.replay()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(replays):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        g.replay()
+        e.record()
+        torch.cuda.synchronize()
+        ts.append(s.elapsed_time(e) / (2 * C))
+    del g, sets, calls
+    torch.cuda.empty_cache()
+    return float(np.median(ts)) * 1e3, C
+
+
 def run_e2e(torch, dg, probs, steps):
     """Same metric through the binding with pinned host buffers and copies in the timed region."""
     host = []
@@ -278,14 +313,21 @@ def run_e2e(torch, dg, probs, steps):
     return ms, h2d, d2h
 
 
-def cpu_baseline(torch, probs, rows=16, budget_s=30.0):
-    """The oracle as it stands, on the first `rows` rows of A against all of B."""
-    import oracle
+def _blas_threads():
     try:
         import threadpoolctl
-        cores = max(i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas")
+        return max(i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas")
     except Exception:
-        cores = len(os.sched_getaffinity(0))
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(torch, probs, W=None, rows=16, budget_s=30.0, full=True):
+    """The oracle as it stands, on the first `rows` rows of A against all of B
+    (the value); `detail` adds the small dense workload on one thread and on
+    all cores, and the contiguous (8 experts) and Zipf masked (256 groups)
+    workloads once each at full size."""
+    import oracle
+    cores = _blas_threads()
     flops = 0.0
     t = 0.0
     done = 0
@@ -303,9 +345,65 @@ def cpu_baseline(torch, probs, rows=16, budget_s=30.0):
         done += 1
         if t > budget_s:
             break
-    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {rows} rows of A x all of B (incl. fp32->UE8M0 pack and dequantisation) "
-                      f"for {done} of 8 problems; {t:.1f} s"}
+    out = {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+           "sample": f"first {rows} rows of A x all of B (incl. fp32->UE8M0 pack and dequantisation) "
+                     f"for {done} of 8 problems; {t:.1f} s"}
+    if not full or W is None:
+        return out
+    detail = {}
+    # dense 128 x 256 x 512 on one thread and on all cores
+    p0 = W.workload0()
+    sfa0, sfb0 = oracle.pack_ue8m0(p0["sfa_f32"]), oracle.pack_ue8m0(p0["sfb_f32"])
+    fl0 = gemm_flops(128, 256, 512)
+
+    def time_c0(reps=20):
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            oracle.fp8_gemm_nt(p0["a"], sfa0, p0["b"], sfb0)
+        return (time.perf_counter() - t0) / reps
+
+    try:
+        import threadpoolctl
+        with threadpoolctl.threadpool_limits(limits=1, user_api="blas"):
+            s1 = time_c0()
+        detail["dense_128x256x512_1thread"] = {"s": s1, "TFLOP/s": fl0 / s1 / 1e12, "cores": 1}
+    except Exception as e:  # no way to limit the BLAS threads: say so
+        detail["dense_128x256x512_1thread"] = {"unavailable": str(e)[:120]}
+    sa = time_c0()
+    detail["dense_128x256x512_all_cores"] = {"s": sa, "TFLOP/s": fl0 / sa / 1e12, "cores": cores}
+    # contiguous, 8 experts x 4096 x 7168, full size, once
+    p2 = W.workload2_t("cuda")
+    h2 = {k: p2[k].cpu().numpy() for k in ("a", "sfa_f32", "b", "sfb_f32", "m_indices")}
+    del p2
+    torch.cuda.empty_cache()
+    sfa2 = oracle.pack_ue8m0(h2["sfa_f32"])
+    sfb2 = oracle.pack_ue8m0(h2["sfb_f32"].reshape(-1, h2["sfb_f32"].shape[-1])).reshape(*h2["sfb_f32"].shape[:-1], -1)
+    t0 = time.perf_counter()
+    oracle.m_grouped_fp8_gemm_nt_contiguous(h2["a"], sfa2, h2["b"], sfb2, h2["m_indices"])
+    s2 = time.perf_counter() - t0
+    rows2 = int((h2["m_indices"] >= 0).sum())
+    detail["contiguous_8x4096x7168_full"] = {"s": s2, "TFLOP/s": gemm_flops(rows2, 4096, 7168) / s2 / 1e12,
+                                             "cores": cores, "rows": rows2}
+    del h2, sfa2, sfb2
+    # masked Zipf, 256 groups x 7168 x 2048, full size, once (pack + GEMM)
+    p4 = W.workload4_t("cuda")
+    h4 = {k: p4[k].cpu().numpy() for k in ("a", "sfa_f32", "b", "sfb_f32")}
+    mm4 = p4["masked_m_host"]
+    del p4
+    torch.cuda.empty_cache()
+    t0 = time.perf_counter()
+    sfa4 = oracle.pack_ue8m0(h4["sfa_f32"].reshape(-1, 16)).reshape(256, 512, -1)
+    sfb4 = oracle.pack_ue8m0(h4["sfb_f32"].reshape(-1, 16)).reshape(256, 56, -1)
+    oracle.m_grouped_fp8_gemm_nt_masked(h4["a"], sfa4, h4["b"], sfb4, mm4)
+    s4 = time.perf_counter() - t0
+    rows4 = int(np.clip(mm4, 0, 512).sum())
+    gnz = int((mm4 > 0).sum())
+    by4 = rows4 * 2048 + gnz * 7168 * 2048 + 2 * rows4 * 7168
+    detail["masked_zipf_256x7168x2048_full"] = {"s": s4, "GB/s": by4 / s4 / 1e9,
+                                                "TFLOP/s": gemm_flops(rows4, 7168, 2048) / s4 / 1e12,
+                                                "cores": cores, "rows": rows4}
+    out["detail"] = detail
+    return out
 
 
 def detail_workloads(torch, W, dg, peaks, reps=8):
@@ -313,10 +411,18 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
     out = {}
     dev = "cuda"
 
+    def settle(seconds=0.4):
+        """Let the SM clock recover before the next workload: a sustained
+        HBM-heavy leg (the masked replays) drives the part into its power cap
+        and the clock stays low for ~0.1 s afterwards."""
+        torch.cuda.synchronize()
+        time.sleep(seconds)
+
     def frac_tensor_mem(fl, by, ms):
         t = ms * 1e-3
         return max(fl / (peaks["fp8"] * 1e12), by / (peaks["hbm"] * 1e9)) / t
 
+    settle()
     # contiguous: 8 experts, N=4096, K=7168
     p = W.workload2_t(dev)
     sfa = dg.pack_ue8m0(p["sfa_f32"])
@@ -339,6 +445,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                      "valid_rows": rows, "M_total": p["M_total"]}
     del p, sfa, sfb, d
 
+    settle()
     # the same experts and row counts without padding, groups given by psum_m
     p = W.psum_t(W.contiguous_counts(), 4096, 7168, seed=1002, device=dev)
     sfa = dg.pack_ue8m0(p["sfa_f32"])
@@ -360,7 +467,15 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor", "rows": rows}
     del p, sfa, sfb, d
 
-    def masked_case(name, p, with_pack, rng):
+    def masked_replays(name, p, with_pack, draw, replays=100, fresh=2):
+        """The masked workloads as stated: the graph holds the masked GEMM (and,
+        with_pack, the UE8M0 pack of the activation scales before it) and
+        nothing else. Before every replay, outside the timed interval, a new
+        masked_m draw is copied in; with_pack also copies in a fresh
+        quantisation of the activations (E4M3 codes and their fp32 scales,
+        cycled from `fresh` seeded sets), which the graph's pack kernel then
+        packs. Each replay is bracketed by its own events; the median and p90
+        over `replays` replays are reported."""
         G, max_m, N, K = p["G"], p["max_m"], p["N"], p["K"]
         kp = kp_of(K)
         sfb = dg.pack_ue8m0(p["sfb_f32"])
@@ -368,25 +483,45 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
         if not with_pack:
             dg.pack_ue8m0(p["sfa_f32"], sfa)
         d = torch.empty((G, max_m, N), dtype=torch.bfloat16, device=dev)
-        # a pool of masked_m draws; each call of the graph copies in the next one
-        draws = [p["masked_m_host"]] + [rng(r) for r in range(1, reps)]
-        pool = torch.from_numpy(np.stack(draws).astype(np.int32)).to(dev)
+        draws = [p["masked_m_host"]] + [draw(r) for r in range(1, replays)]
+        mm_pool = torch.from_numpy(np.stack(draws).astype(np.int32)).to(dev)
+        act_pool = []
+        if with_pack:
+            act_pool.append((p["a"].clone(), p["sfa_f32"].clone()))
+            g = torch.Generator(device=dev)
+            for f in range(1, fresh):
+                g.manual_seed(7000 + f)
+                qa, qs = W.quantise_rows_t(torch.randn((G * max_m, K), generator=g, device=dev))
+                act_pool.append((qa.view(G, max_m, K), qs.view(G, max_m, K // 128)))
         mm = p["masked_m"]
-        ops = []
-        for r in range(reps):
-            def op(r=r):
-                mm.copy_(pool[r])
-                if with_pack:
-                    dg.pack_ue8m0(p["sfa_f32"], sfa)
-                dg.m_grouped_fp8_gemm_nt_masked(p["a"], sfa, p["b"], sfb, d, mm)
-            ops.append(op)
-        ops[0]()
+
+        def call():
+            if with_pack:
+                dg.pack_ue8m0(p["sfa_f32"], sfa)
+            dg.m_grouped_fp8_gemm_nt_masked(p["a"], sfa, p["b"], sfb, d, mm)
+
+        settle()
+        call()
         torch.cuda.synchronize()
-        g = EventGraph(ops)
-        g.replay()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            call()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+        for r in range(3):  # warm-up replays
+            graph.replay()
         torch.cuda.synchronize()
-        durs = g.durations_ms()
-        g.close()
+        for r in range(replays):
+            mm.copy_(mm_pool[r])
+            if with_pack:
+                qa, qs = act_pool[r % len(act_pool)]
+                p["a"].copy_(qa)
+                p["sfa_f32"].copy_(qs)
+            evs[r][0].record()
+            graph.replay()
+            evs[r][1].record()
+        torch.cuda.synchronize()
+        durs = [a.elapsed_time(b) for a, b in evs]
+        del graph
         gbs, fr = [], []
         for r, ms in enumerate(durs):
             m = np.clip(draws[r], 0, max_m)
@@ -397,20 +532,31 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                 by += G * max_m * (K // 128) * 4 + G * max_m * kp * 4
             gbs.append(by / ms / 1e6)
             fr.append(by / (peaks["hbm"] * 1e9) / (ms * 1e-3))
-        out[name] = {"us": statistics.median(durs) * 1e3, "GB/s": statistics.median(gbs),
-                     "roofline_frac": statistics.median(fr), "bound": "hbm", "calls": reps,
-                     "with_pack": with_pack}
+        tr = committed_traffic(name)
+        traffic = None if tr is None else {"dram_bytes": tr["dram_bytes"], "algorithmic_bytes": tr["algorithmic_bytes"],
+                                           "ratio": tr["dram_bytes"] / tr["algorithmic_bytes"],
+                                           "of": "the first replay's masked_m draw (ncu, one launch)"}
+        out[name] = {"us": float(np.median(durs)) * 1e3, "us_p90": float(np.percentile(durs, 90)) * 1e3, "traffic": traffic,
+                     "GB/s": float(np.median(gbs)), "roofline_frac": float(np.median(fr)),
+                     "roofline_frac_p10": float(np.percentile(fr, 10)), "bound": "hbm", "replays": replays,
+                     "with_pack": with_pack,
+                     "protocol": "plain graph (pack + GEMM, or GEMM); fresh masked_m"
+                                 + (" and fresh activations + fp32 scales" if with_pack else "")
+                                 + " copied in before each replay, outside its events"}
 
+    settle()
     for proj in ("up", "down"):
         p = W.workload3_t(proj, dev)
-        masked_case(f"masked_decode_32g_{proj}_{p['N']}x{p['K']}", p, False,
-                    lambda r: W.masked_m_uniform(W.rng_for(5000 + r)))
+        masked_replays(f"masked_decode_32g_{proj}_{p['N']}x{p['K']}", p, False,
+                       lambda r: W.masked_m_uniform(W.rng_for(5000 + r)))
         del p
+    settle()
     p = W.workload4_t(dev)
-    masked_case("masked_zipf_256g_7168x2048_pack+gemm", p, True,
-                lambda r: W.zipf_masked_m(W.rng_for(6000 + r)))
+    masked_replays("masked_zipf_256g_7168x2048_pack+gemm", p, True, lambda r: W.zipf_masked_m(W.rng_for(6000 + r)))
     del p
+    torch.cuda.empty_cache()
 
+    settle()
     # dense with an accumulation matrix: D (fp32) = C (fp32) + A.B^T, in place
     M, N, K = 4096, 7168, 16384
     p = W.workload1_t(M, N, K, dev)
@@ -429,6 +575,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                                  "roofline_frac": frac_tensor_mem(fl, by, ms), "bound": "tensor"}
     del p, sfa, sfb, d
 
+    settle()
     # other operand layouts (A stored [K, M] and/or B stored [K, N]), 4096x7168x16384
     M, N, K = 4096, 7168, 16384
     p = W.workload1_t(M, N, K, dev)
@@ -439,6 +586,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
     for name, fn, a_op, b_op in (("nn", dg.fp8_gemm_nn, p["a"], b_kn), ("tn", dg.fp8_gemm_tn, a_km, b_kn),
                                  ("tt", dg.fp8_gemm_tt, a_km, p["b"])):
         op = lambda fn=fn, a_op=a_op, b_op=b_op: fn(a_op, sfa, b_op, sfb, d)
+        settle()
         op()
         g = EventGraph([op] * 4)
         g.replay()
@@ -452,6 +600,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
     # the same NT problem with one weight scale row per row of B (sfb [N, KP])
     sfb_rows = sfb.repeat_interleave(128, dim=0)[:N].contiguous()
     op = lambda: dg.fp8_gemm_nt_sfb_gran(p["a"], sfa, p["b"], sfb_rows, d, 1)
+    settle()
     op()
     g = EventGraph([op] * 4)
     g.replay()
@@ -464,6 +613,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                               "bound": "tensor"}
     del p, sfa, sfb, sfb_rows, d, a_km, b_kn
 
+    settle()
     # per-token FP8 quantiser: bf16 activations [4096, 7168] -> E4M3 + packed UE8M0
     rows, K = 4096, 7168
     x = torch.randn((rows, K), device=dev).to(torch.bfloat16)
@@ -482,6 +632,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                                                   "bound": "hbm"}
     del x, qb, sp
 
+    settle()
     # BF16 masked decode (same shapes and masked_m draws, plain bf16 operands)
     def masked_bf16_case(name, q, rng):
         G, max_m, N, K = q["G"], q["max_m"], q["N"], q["K"]
@@ -495,6 +646,7 @@ def detail_workloads(torch, W, dg, peaks, reps=8):
                 mm.copy_(pool[r])
                 dg.m_grouped_bf16_gemm_nt_masked(q["a"], q["b"], d, mm)
             ops.append(op)
+        settle()
         ops[0]()
         torch.cuda.synchronize()
         g = EventGraph(ops)
@@ -589,24 +741,19 @@ def run_ours(args):
     dom = int(np.argmax(mean_gemm))
     M, N, K = shapes()[dom]
     achieved = gemm_flops(M, N, K) / (mean_gemm[dom] * 1e-3) / 1e12
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "dense_gemm_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            with open(tpath) as f:
-                tj = json.load(f)
-            key = f"{M}x{N}x{K}"
-            traffic = tj.get(key) if tj.get("kernel_rev") == dg_kernel_rev() else None
-        except Exception:
-            traffic = None
+    traffic = committed_traffic(f"dense_{M}x{N}x{K}")
+    traffic = traffic["dram_bytes"] if traffic else None
     per_shape = {}
     for i, (m, n, k) in enumerate(shapes()):
-        t = mean_gemm[i] * 1e-3
+        us, copies = steady_state_us(torch, dg, probs[i])
+        t = us * 1e-6
+        t_step = mean_gemm[i] * 1e-3
         fl, by = gemm_flops(m, n, k), dense_bytes(m, n, k)
+        roof = max(fl / (peaks["fp8"] * 1e12), by / (peaks["hbm"] * 1e9))
         per_shape[f"{m}x{n}x{k}"] = {
-            "us": mean_gemm[i] * 1e3, "TFLOP/s": fl / t / 1e12, "GB/s": by / t / 1e9,
-            "roofline_frac": max(fl / (peaks["fp8"] * 1e12), by / (peaks["hbm"] * 1e9)) / t,
+            "us": us, "TFLOP/s": fl / t / 1e12, "GB/s": by / t / 1e9, "roofline_frac": roof / t,
             "bound": "tensor" if fl / (peaks["fp8"] * 1e12) > by / (peaks["hbm"] * 1e9) else "hbm",
+            "us_in_step": t_step * 1e6, "roofline_frac_in_step": roof / t_step, "input_copies": copies,
         }
     launches = len(ops) * args.steps
     per_launch.close()
@@ -623,6 +770,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD, "shapes": [list(sh) for sh in shapes()],
                        "l2": "inputs larger than L2 (step footprint ~1.2 GB, each buffer reused only after all others)",
                        "timing": "K steps in one CUDA graph (kernels only); per-kernel times from a second replay with an event node after every launch",
+                       "per_shape": "us: per call in a graph of back-to-back calls of one shape over input copies totalling >= 4x L2 (programmatic dependent launch overlaps each call's start with the previous call's end); us_in_step: the step's replay with an event node after every launch (each launch then pays its own start-up)",
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["fp8"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["fp8"], "traffic": traffic,
@@ -638,7 +786,7 @@ def run_ours(args):
         }
         if not args.no_detail:
             result["detail"] = detail_workloads(torch, W, dg, peaks)
-        result["cpu_baseline"] = cpu_baseline(torch, probs)
+        result["cpu_baseline"] = cpu_baseline(torch, probs, W, full=not args.no_detail)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -648,6 +796,20 @@ def run_ours(args):
     if dev_err:
         log(f"device status word = {dev_err}")
         sys.exit(1)
+
+
+def committed_traffic(key):
+    """The DRAM bytes of one launch from the committed ncu record
+    (profiles/traffic.json), only while the kernel sources hash to the revision
+    the counters were taken on; else None."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            tj = json.load(f)
+    except Exception:
+        return None
+    if tj.get("kernel_rev") != dg_kernel_rev():
+        return None
+    return tj.get(key)
 
 
 def dg_kernel_rev():
@@ -693,11 +855,7 @@ def run_reference(args):
     for _ in range(args.steps):
         fl += step()
     dt = time.perf_counter() - t0
-    try:
-        import threadpoolctl
-        cores = max(i["num_threads"] for i in threadpoolctl.threadpool_info() if i.get("user_api") == "blas")
-    except Exception:
-        cores = len(os.sched_getaffinity(0))
+    cores = _blas_threads()
     value = fl / dt / 1e12
     sample = f"per step: first {rows} rows of A x first {cols} rows of B for each of the 8 problems (full K)"
     print(json.dumps({

@@ -110,9 +110,20 @@ def _masked_replays(p, with_pack, draws, what):
         assert np.array_equal(_host(sfa), _pack_host(p["sfa_f32"])), "packed activation scales differ"
     for it, m_draw in enumerate(draws):
         mm.copy_(torch.from_numpy(m_draw.astype(np.int32)))
+        if with_pack and it > 0:
+            # a fresh quantisation of the activations, copied into the captured
+            # buffers; the graph's pack kernel packs its scales
+            gen = torch.Generator(device="cuda")
+            gen.manual_seed(900 + it)
+            qa, qs = W.quantise_rows_t(torch.randn((G * max_m, K), generator=gen, device="cuda"))
+            p["a"].copy_(qa.view(G, max_m, K))
+            p["sfa_f32"].copy_(qs.view(G, max_m, K // 128))
+            del qa, qs
         fill_sentinel(d)
         g.replay()
         torch.cuda.synchronize()
+        if with_pack:
+            assert np.array_equal(_host(sfa), _pack_host(p["sfa_f32"])), f"{what} replay {it}: packed scales differ"
         m_clamped = np.clip(m_draw, 0, max_m)
         invalid = torch.from_numpy(np.arange(max_m)[None, :] >= m_clamped[:, None]).cuda()
         assert (d.view(torch.int16)[invalid] == SENT).all().item(), f"{what}: a row past masked_m was written"
@@ -139,6 +150,7 @@ def test_masked_decode_full_size_graph_replay(proj):
 
 
 def test_masked_zipf_full_size_pack_and_gemm_graph():
+    # replays with fresh masked_m and, from the second on, fresh activations and scales
     p = W.workload4_t()
-    draws = [p["masked_m_host"], W.zipf_masked_m(W.rng_for(79))]
+    draws = [p["masked_m_host"], W.zipf_masked_m(W.rng_for(79)), W.zipf_masked_m(W.rng_for(80))]
     _masked_replays(p, True, draws, "masked zipf")
