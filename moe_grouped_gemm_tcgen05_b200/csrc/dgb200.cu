@@ -51,10 +51,10 @@ struct DeviceState {
     std::atomic<bool> ready{false};  // set (release) once every field below is filled
     int sms = 0;
     uint32_t* status = nullptr;  // address of g_dg_device_status on this device
-    int max_pairs[64] = {};      // co-resident CTA pairs per kernel entry (cluster kernels only)
+    int max_pairs[80] = {};      // co-resident CTA pairs per kernel entry (cluster kernels only)
     // co-resident clusters of s CTAs (s = 2..8) per kernel entry, for the
     // cluster split-K of the dense single-CTA kernels (0: not launchable)
-    int max_clusters[64][kMaxClusterSplits + 1] = {};
+    int max_clusters[80][kMaxClusterSplits + 1] = {};
     // fp8_gemm_nt_noalloc only: split-K scratch in the library's static arrays
     float* split_ws = nullptr;
     uint32_t* split_counters = nullptr;
@@ -137,17 +137,19 @@ const KernelEntry kKernels[] = {
     DG_ALL_KINDS(64),  DG_ALL_KINDS(96),  DG_ALL_KINDS(128), DG_ALL_KINDS(160),
     DG_ALL_KINDS(192), DG_ALL_KINDS(224), DG_ALL_KINDS(256),
     DG_ENTRY(128, dg::kDense, 2), DG_ENTRY(160, dg::kDense, 2), DG_ENTRY(192, dg::kDense, 2),
-    DG_ENTRY(224, dg::kDense, 2), DG_ENTRY(256, dg::kDense, 2),
+    DG_ENTRY(224, dg::kDense, 2), DG_ENTRY(240, dg::kDense, 2), DG_ENTRY(256, dg::kDense, 2),
     DG_ENTRY(128, dg::kContiguous, 2), DG_ENTRY(160, dg::kContiguous, 2), DG_ENTRY(192, dg::kContiguous, 2),
     DG_ENTRY(224, dg::kContiguous, 2), DG_ENTRY(256, dg::kContiguous, 2),
     DG_BF16_MASKED(64), DG_BF16_MASKED(96), DG_BF16_MASKED(128), DG_BF16_MASKED(160),
     DG_BF16_MASKED(192), DG_BF16_MASKED(224), DG_BF16_MASKED(256),
     DG_LAYOUT(128, 1), DG_LAYOUT(256, 1), DG_LAYOUT(128, 2), DG_LAYOUT(256, 2), DG_LAYOUT(128, 3), DG_LAYOUT(256, 3),
     DG_ACC(64, 1), DG_ACC(96, 1), DG_ACC(128, 1), DG_ACC(160, 1), DG_ACC(192, 1), DG_ACC(224, 1), DG_ACC(256, 1),
-    DG_ACC(128, 2), DG_ACC(160, 2), DG_ACC(192, 2), DG_ACC(224, 2), DG_ACC(256, 2),
+    DG_ACC(128, 2), DG_ACC(160, 2), DG_ACC(192, 2), DG_ACC(224, 2), DG_ACC(240, 2), DG_ACC(256, 2),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
-constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 256};
+// 240 (a 16-column tail chunk, double-buffered at nearly 256 columns) is built
+// for the dense form on CTA pairs only
+constexpr int kBlockNs[] = {64, 96, 128, 160, 192, 224, 240, 256};
 
 // ------------------------------------------------------------------ init ----
 
@@ -169,7 +171,7 @@ dg_status setup_device(int dev, DeviceState& st) {
         return DG_ERR_CUDA;
     if (major != 10 || minor != 0) return DG_ERR_UNSUPPORTED;  // built for sm_100a only
     if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DG_ERR_CUDA;
-    static_assert(kNumKernels <= 64, "DeviceState::max_pairs too small");
+    static_assert(kNumKernels <= 80, "DeviceState::max_pairs too small");
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
         if (cudaFuncSetAttribute(e.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, e.smem) != cudaSuccess)
@@ -355,7 +357,11 @@ double kblock_clocks(int bn, int cg, int rows_a) {
     return tc > l2 ? tc : l2;
 }
 
-int num_acc_for(int bn) { return (2 * bn + 2 * (4 + 4 * ((bn + 127) / 128)) <= 512) ? 2 : 1; }
+// Accumulator slots in TMEM (the kernel's GemmConfig::NUM_ACC).
+int num_acc_for(int bn) {
+    if (bn % 32 != 0) return 2;  // slots on 256-column boundaries, scale sets in the tails
+    return (2 * bn + 2 * (4 + 4 * ((bn + 127) / 128)) <= 512) ? 2 : 1;
+}
 
 struct TileChoice {
     const KernelEntry* entry;

@@ -144,7 +144,8 @@ __host__ __device__ constexpr int sched_ints() {
 
 template <int BN, int CG, int SCHED_INTS, int DT = kE4M3>
 struct GemmConfig {
-    static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 32 in [32, 256]");
+    static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 16 in [32, 256]");
+    static_assert(BN % 32 == 0 || CG == 2, "tiles with a 16-column tail chunk are built for CTA pairs");
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
     static constexpr int B_ROWS = BN / CG;                      // rows of B in this CTA's shared memory
     static constexpr int A_BYTES = BM * BK;
@@ -165,15 +166,23 @@ struct GemmConfig {
     static_assert(STAGES >= 2, "pipeline too shallow");
     static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES;
 
-    // TMEM columns: accumulator slot(s) of BN columns, then two sets of scale
+    // TMEM columns: accumulator slot(s) of BN columns and two sets of scale
     // columns (4 of A scales and 4 per 128-column chunk of B scales), used by
     // alternate groups so that the copy of the next group's scales never
-    // overwrites words that MMAs still in the pipe are reading.
+    // overwrites words that MMAs still in the pipe are reading. Widths that are
+    // multiples of 32 put the slots side by side and the scale sets after them;
+    // a width with a 16-column tail (BN = 240) keeps each slot on a 256-column
+    // boundary and puts one scale set in the 16 columns after each slot.
     static constexpr int ACC_COLS = BN;
     static constexpr int SF_COLS = DT == kE4M3 ? 4 + 4 * SFB_CHUNKS : 0;
-    static constexpr int NUM_ACC = (2 * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1;
-    static constexpr int SF_BASE = NUM_ACC * ACC_COLS;
-    static_assert(SF_BASE + 2 * SF_COLS <= 512, "TMEM overflow");
+    static constexpr bool TAIL16 = BN % 32 != 0;
+    static constexpr int ACC_STRIDE = TAIL16 ? 256 : BN;   // columns between accumulator slots
+    static constexpr int NUM_ACC =
+        TAIL16 ? ((256 - BN >= SF_COLS) ? 2 : 1) : ((2 * ACC_COLS + 2 * SF_COLS <= 512) ? 2 : 1);
+    static constexpr int SF_SET0 = TAIL16 ? BN : NUM_ACC * ACC_COLS;
+    static constexpr int SF_SET1 = TAIL16 ? 256 + BN : SF_SET0 + SF_COLS;
+    static_assert(SF_SET1 + SF_COLS <= 512, "TMEM overflow");
+    static_assert(!TAIL16 || NUM_ACC == 2, "a 16-column-tail tile is double-buffered");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC = DT == kE4M3 ? idesc_mxf8_e4m3_ue8m0(BM * CG, BN) : idesc_bf16_f32(BM * CG, BN);
     // K values per 128-byte row of a stage and per MMA instruction
@@ -1058,8 +1067,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // the current group's first K-block is issued, so that wait and
             // copy overlap MMAs already queued (the tensor pipe runs a thread's
             // copies and MMAs in issue order).
-            uint32_t sf_cur = tmem_base + Cfg::SF_BASE;
-            uint32_t sf_nxt = sf_cur + Cfg::SF_COLS;
+            uint32_t sf_cur = tmem_base + Cfg::SF_SET0;
+            uint32_t sf_nxt = tmem_base + Cfg::SF_SET1;
             // next group's scale words (both CTAs of a pair) -> TMEM at `dst`;
             // the ring slot is free again once the copy has completed
             auto copy_scales = [&](uint32_t dst) -> bool {
@@ -1083,7 +1092,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                  t += units) {
                 if (!wait_warp(&tempty_bar[acc], acc_phase ^ 1u, p, s_abort)) { aborted = true; break; }
                 tc_fence_after();  // the epilogue's TMEM reads precede the MMAs below
-                const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
+                const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_STRIDE;
                 // the tile's first group: its scales go to the set the previous
                 // group did not use
                 if (!copy_scales(sf_nxt)) { aborted = true; break; }
@@ -1204,7 +1213,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             const bool use_tma = (KIND == kDense) ? true : (__all_sync(0xffffffffu, valid) != 0);
             if (!wait_warp(&tfull_bar[acc], acc_phase, p, s_abort)) break;
             tc_fence_after();
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_COLS;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * Cfg::ACC_STRIDE;
             const int n0 = c.n_blk * BN;
             __nv_bfloat16* drow = p.d + out_row * static_cast<size_t>(p.n) + n0;
             constexpr int kMaxBatch = 128;
@@ -1359,14 +1368,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                                 make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
                 }
             };
+            // the 16-column tail chunk of a 240-wide tile (pairs, dense form):
+            // fp32 -> bf16 (or + C, fp32) with direct 16-byte stores of the valid rows
+            auto emit16 = [&](const uint32_t* v, int hc) {
+                const int col = n0 + hc;
+                if (col >= p.n || !valid) return;  // N % 8 == 0: 8-column pieces are wholly in or out
+                float f[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) f[i] = __uint_as_float(v[i]);
+                const size_t at = out_row * static_cast<size_t>(p.n) + col;
+                if constexpr (EPI == 1) {
+                    if (p.c != nullptr) {
+                        if (p.out_f32) {
+                            const float* crow = static_cast<const float*>(p.c) + at;
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                if (col + 4 * q4 >= p.n) continue;
+                                const float4 x = *reinterpret_cast<const float4*>(crow + 4 * q4);
+                                f[4 * q4] += x.x; f[4 * q4 + 1] += x.y; f[4 * q4 + 2] += x.z; f[4 * q4 + 3] += x.w;
+                            }
+                        } else {
+                            const __nv_bfloat16* crow = static_cast<const __nv_bfloat16*>(p.c) + at;
+#pragma unroll
+                            for (int q8 = 0; q8 < 2; ++q8) {
+                                if (col + 8 * q8 >= p.n) continue;
+                                const uint4 x = *reinterpret_cast<const uint4*>(crow + 8 * q8);
+                                const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                                for (int h2 = 0; h2 < 4; ++h2) {
+                                    const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                                    f[8 * q8 + 2 * h2] += c2.x;
+                                    f[8 * q8 + 2 * h2 + 1] += c2.y;
+                                }
+                            }
+                        }
+                    }
+                    if (p.out_f32) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            if (col + 4 * q4 < p.n)
+                                *reinterpret_cast<float4*>(p.d32 + at + 4 * q4) =
+                                    make_float4(f[4 * q4], f[4 * q4 + 1], f[4 * q4 + 2], f[4 * q4 + 3]);
+                        return;
+                    }
+                }
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+                    w[i] = *reinterpret_cast<uint32_t*>(&b2);
+                }
+#pragma unroll
+                for (int q8 = 0; q8 < 2; ++q8)
+                    if (col + 8 * q8 < p.n)
+                        *reinterpret_cast<uint4*>(p.d + at + 8 * q8) =
+                            make_uint4(w[4 * q8], w[4 * q8 + 1], w[4 * q8 + 2], w[4 * q8 + 3]);
+            };
             if (emit_tile && !(kCanSplit && split)) {
 #pragma unroll
                 for (int h = 0; h < BN; h += 128) {
                     const int cols = (BN - h) < kMaxBatch ? (BN - h) : kMaxBatch;  // compile-time after unrolling
                     uint32_t r[kMaxBatch];
 #pragma unroll
-                    for (int j = 0; j < kMaxBatch / 32; ++j)
-                        if (32 * j < cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
+                    for (int j = 0; j < kMaxBatch / 32; ++j) {
+                        if (32 * j + 32 <= cols) tmem_ld_32x32b_x32(taddr + h + 32 * j, r + 32 * j);
+                        else if (32 * j < cols) tmem_ld_32x32b_x16(taddr + h + 32 * j, r + 32 * j);
+                    }
                     tc_wait_ld();
                     if (h + 128 >= BN) {
                         // last TMEM read of this accumulator: hand it back to the MMA warp
@@ -1378,8 +1445,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         }
                     }
 #pragma unroll
-                    for (int j = 0; j < kMaxBatch / 32; ++j)
-                        if (32 * j < cols) emit32(r + 32 * j, h + 32 * j);
+                    for (int j = 0; j < kMaxBatch / 32; ++j) {
+                        if (32 * j + 32 <= cols) emit32(r + 32 * j, h + 32 * j);
+                        else if (32 * j < cols) emit16(r + 32 * j, h + 32 * j);
+                    }
                 }
             }
             if constexpr (kCanSplit) {

@@ -53,6 +53,7 @@ CONFIGS = [  # (M, N, K, bn, cg, splits)
     (300, 400, 1024, 0, 0, 0),
     (257, 264, 640, 128, 1, 1),
     (512, 1000, 2048, 224, 2, 1),    # CTA pairs
+    (300, 776, 1024, 240, 2, 1),     # CTA pairs, 240-wide tiles (16-column tail chunk)
     (64, 2112, 4096, 64, 1, 4),      # split-K (8 K groups)
     (1, 520, 512, 0, 0, 0),
 ]

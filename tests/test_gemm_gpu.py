@@ -64,10 +64,12 @@ def test_dense_parity_every_tile_width(bn, mnk):
 
 
 PAIR_BLOCK_NS = [128, 160, 192, 224, 256]
+DENSE_PAIR_BLOCK_NS = PAIR_BLOCK_NS + [240]   # 240: a 16-column tail chunk, dense pairs only
 
 
-@pytest.mark.parametrize("bn", PAIR_BLOCK_NS)
-@pytest.mark.parametrize("mnk", [(300, 400, 1024), (512, 256, 512), (257, 264, 640), (1024, 1000, 2048)])
+@pytest.mark.parametrize("bn", DENSE_PAIR_BLOCK_NS)
+@pytest.mark.parametrize("mnk", [(300, 400, 1024), (512, 256, 512), (257, 264, 640), (1024, 1000, 2048),
+                                 (512, 776, 1024)])
 def test_dense_parity_cta_pairs(bn, mnk):
     # 256-row tiles on CTA pairs; M not a multiple of 256 leaves the odd CTA
     # of the last pair partly or wholly past M
@@ -105,7 +107,7 @@ def _pack_bytes_host(byts):
     return w.astype(np.uint32).view(np.int32)
 
 
-@pytest.mark.parametrize("bn,cg", [(b, 1) for b in BLOCK_NS] + [(b, 2) for b in PAIR_BLOCK_NS])
+@pytest.mark.parametrize("bn,cg", [(b, 1) for b in BLOCK_NS] + [(b, 2) for b in DENSE_PAIR_BLOCK_NS])
 def test_one_hot_rows_are_bit_exact(bn, cg):
     # one-hot A rows with power-of-two scales: every output is a single product
     # e4m3 * 2^a * 2^b, exactly representable in bf16

@@ -89,6 +89,7 @@ def _ref_dense(p):
 # pairs whose odd CTA is partly or wholly past M, and split-K
 DENSE_CASES = [((200, 776, 2560), 128, 1, 1), ((200, 776, 2560), 256, 1, 1), ((77, 264, 1024), 96, 1, 1),
                ((300, 400, 1024), 160, 2, 1), ((129, 520, 1536), 256, 2, 1), ((1, 136, 1024), 224, 1, 1),
+               ((300, 776, 1024), 240, 2, 1), ((257, 496, 1024), 240, 2, 1),
                ((64, 776, 4096), 128, 1, 4), ((200, 264, 2560), 64, 1, 3), ((130, 1000, 3200), 256, 1, 2)]
 
 
@@ -107,6 +108,7 @@ def test_dense_stays_inside_d(mnk, bn, cg, splits):
 
 @pytest.mark.parametrize("out_f32", [False, True])
 @pytest.mark.parametrize("mnk,bn,cg,splits", [((200, 776, 2560), 128, 1, 1), ((300, 400, 1024), 192, 2, 1),
+                                             ((300, 776, 1024), 240, 2, 1),
                                              ((64, 520, 4096), 128, 1, 4)])
 def test_accumulate_epilogue_stays_inside_d(mnk, bn, cg, splits, out_f32):
     M, N, K = mnk

@@ -19,6 +19,7 @@ pytestmark = pytest.mark.gpu
 
 BLOCK_NS = [64, 96, 128, 160, 192, 224, 256]
 PAIR_BLOCK_NS = [128, 160, 192, 224, 256]
+DENSE_PAIR_BLOCK_NS = PAIR_BLOCK_NS + [240]   # 240: dense pairs only
 
 
 @pytest.fixture(autouse=True)
@@ -67,7 +68,7 @@ def test_dense_every_tile_width(bn, mnk):
     check_fp(bf16_to_f64(d), _ref(p), f"per-row B scales {mnk} bn={bn}")
 
 
-@pytest.mark.parametrize("bn", PAIR_BLOCK_NS)
+@pytest.mark.parametrize("bn", DENSE_PAIR_BLOCK_NS)
 def test_dense_cta_pairs(bn):
     p = W.dense(300, 520, 1024, seed=bn, sfb_gran_n=1)
     d = _dense(p, bn, cg=2)
@@ -92,7 +93,7 @@ def test_dense_with_c(out):
     check_fp(got, _ref(p, c=c_vals), f"per-row B scales, C, {out}")
 
 
-@pytest.mark.parametrize("bn,cg", [(b, 1) for b in BLOCK_NS] + [(b, 2) for b in PAIR_BLOCK_NS])
+@pytest.mark.parametrize("bn,cg", [(b, 1) for b in BLOCK_NS] + [(b, 2) for b in DENSE_PAIR_BLOCK_NS])
 def test_one_hot_rows_are_bit_exact(bn, cg):
     # one-hot A rows, power-of-two scales, a different scale row for every row
     # of B: each output is one product e4m3 * 2^a * 2^b, exact in bf16
