@@ -760,9 +760,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     // Everything above touches only this CTA's shared memory, TMEM and the
     // kernel parameters; global memory (operands, scales, metadata, status,
     // split-K scratch) is read or written only after the grids this launch
-    // depends on have completed. The next launch may start right away.
-    griddep_wait();
+    // depends on have completed. The next launch in the stream may be
+    // scheduled right away (it waits for this grid in turn).
     griddep_launch_dependents();
+    griddep_wait();
     if constexpr (KIND == kMasked) {
         // masked_m clamped to [0, max_m]
         for (int g = threadIdx.x; g < p.groups; g += NUM_THREADS) s_mm[g] = min(max(__ldg(p.meta + g), 0), p.rows);

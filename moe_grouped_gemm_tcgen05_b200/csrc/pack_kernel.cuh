@@ -21,8 +21,8 @@ __device__ __forceinline__ uint32_t ue8m0_byte(float x) {
 // cols % 4 == 0 and 16-byte aligned input: word i packs floats 4i..4i+3, so the
 // whole tensor is one flat stream of float4 -> int32.
 __global__ void pack_ue8m0_vec4_kernel(const float4* __restrict__ sf, uint32_t* __restrict__ out, int64_t words) {
-    griddep_wait();
     griddep_launch_dependents();
+    griddep_wait();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
         const float4 v = __ldg(sf + i);
@@ -33,8 +33,8 @@ __global__ void pack_ue8m0_vec4_kernel(const float4* __restrict__ sf, uint32_t* 
 // General layout: rows x cols floats -> rows x kp words, zero bytes past cols.
 __global__ void pack_ue8m0_rows_kernel(const float* __restrict__ sf, uint32_t* __restrict__ out, int64_t rows,
                                        int cols, int kp) {
-    griddep_wait();
     griddep_launch_dependents();
+    griddep_wait();
     const int64_t words = rows * kp;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words; i += stride) {
@@ -53,8 +53,8 @@ __global__ void pack_ue8m0_rows_kernel(const float* __restrict__ sf, uint32_t* _
 
 // Counts scales whose sign bit is set or whose mantissa is non-zero.
 __global__ void pack_ue8m0_validate_kernel(const float* __restrict__ sf, int64_t n, int32_t* __restrict__ bad) {
-    griddep_wait();
     griddep_launch_dependents();
+    griddep_wait();
     int local = 0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
@@ -119,8 +119,8 @@ __global__ void __launch_bounds__(QUANT_THREADS, QUANT_BLOCKS_PER_SM)
 quantize_fp8_1x128_kernel(const void* __restrict__ x, uint32_t* __restrict__ q,
                                           uint8_t* __restrict__ sf_bytes, float* __restrict__ sf_f32, int64_t rows,
                                           int kb, int kp) {
-    griddep_wait();
     griddep_launch_dependents();
+    griddep_wait();
     const int lane = static_cast<int>(threadIdx.x & 31u);
     const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
