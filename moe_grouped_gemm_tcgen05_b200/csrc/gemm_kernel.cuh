@@ -671,17 +671,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT>;
     // instruction descriptor with the operands' major modes
     constexpr uint32_t kIdesc = Cfg::IDESC | (kMnA ? (1u << 15) : 0u) | (kMnB ? (1u << 16) : 0u);
-    // MN-major descriptor strides: one atom is 128 K-rows x 128 bytes
+    // MN-major descriptor strides: one atom is 128 K-rows x 128 bytes of M or
+    // N (one TMA box); groups of 8 K-rows are 1024 bytes apart (stride byte
+    // offset), and consecutive atoms along M or N 16 KB apart (leading byte
+    // offset), so one MMA reads a whole 256-column MN-major B tile (two atoms).
     constexpr uint32_t kMnAtomBytes = BK * 128;
-    // Every MMA reads a single atom of an MN-major operand (A tiles are 128
-    // rows; an MN-major B tile is issued one 128-column atom at a time), so the
-    // stride between atoms along MN is never used; both offsets are set to the
-    // 1024-byte stride between groups of 8 K-rows.
-    constexpr uint32_t kMnLbo = 8 * 128;
+    constexpr uint32_t kMnLbo = kMnAtomBytes;
     constexpr uint32_t kMnSbo = 8 * 128;
-    constexpr int kBParts = kMnB ? BN / 128 : 1;   // MMAs per K-step along N
-    constexpr uint32_t kIdescPart = kMnB ? (idesc_mxf8_e4m3_ue8m0(BM * CG, 128) | (kMnA ? (1u << 15) : 0u) | (1u << 16))
-                                         : kIdesc;
     constexpr int STAGES = Cfg::STAGES;
     constexpr int NUM_ACC = Cfg::NUM_ACC;
 
@@ -1129,17 +1125,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                                 const uint64_t koff = static_cast<uint64_t>((k * 32) >> 4);
                                 const uint64_t koff_mn = static_cast<uint64_t>((k * 32 * 128) >> 4);
                                 const uint32_t accumulate = (gi > c.kg0 || kb > kb0 || k > 0) ? 1u : 0u;
-                                if constexpr (DT == kE4M3 && kBParts > 1) {
-                                    // MN-major B: one N = 128 MMA per atom, into its
-                                    // accumulator columns, with its chunk of B scales
-#pragma unroll
-                                    for (int part = 0; part < kBParts; ++part)
-                                        tc_mma_mxf8f6f4_block_scale<CG>(
-                                            d_tmem + 128 * part, adesc + (kMnA ? koff_mn : koff),
-                                            bdesc + ((part * kMnAtomBytes) >> 4) + koff_mn,
-                                            idesc_with_sf_id(kIdescPart, sf_id), sfa_t,
-                                            (sf_cur + 4 + 4 * part) | (sf_id << 30), accumulate);
-                                } else if constexpr (DT == kE4M3)
+                                if constexpr (DT == kE4M3)
                                     tc_mma_mxf8f6f4_block_scale<CG>(d_tmem, adesc + (kMnA ? koff_mn : koff),
                                                                     bdesc + (kMnB ? koff_mn : koff), idesc, sfa_t,
                                                                     sfb_t, accumulate);
