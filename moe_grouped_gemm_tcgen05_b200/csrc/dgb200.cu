@@ -102,9 +102,9 @@ const bool g_sf_vec4 = [] {
 
 // --------------------------------------------------------------- kernels ----
 
-template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0>
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0, int AR = dg::BM>
 void* kernel_ptr() {
-    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT, LAYOUT, EPI>);
+    return reinterpret_cast<void*>(&dg::fp8_block_scaled_gemm_kernel<BN, KIND, CG, DT, LAYOUT, EPI, AR>);
 }
 
 struct KernelEntry {
@@ -114,16 +114,20 @@ struct KernelEntry {
     int dt;      // operand type (dg::kE4M3 block-scaled, dg::kBF16)
     int layout;  // dense: bit 0 A stored [K, M], bit 1 B stored [K, N]
     int epi;     // dense: 1 = epilogue of D = C + A.B^T (bf16 or fp32 D)
+    int a_rows;  // rows of A per stage: 128, or 64 (dense, M <= 64)
     void* fn;
     int smem;
     int stages;       // depth of the operand ring
     int stage_bytes;  // bytes of one stage (A and B tiles)
 };
 
-#define DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, EPI)                                                             \
-    {BN, KIND, CG, DT, LAYOUT, EPI, kernel_ptr<BN, KIND, CG, DT, LAYOUT, EPI>(),                                \
-     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::SMEM_BYTES, dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGES, \
-     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT>::STAGE_BYTES}
+#define DG_ENTRY_TLEA(BN, KIND, CG, DT, LAYOUT, EPI, AR)                                                        \
+    {BN, KIND, CG, DT, LAYOUT, EPI, AR, kernel_ptr<BN, KIND, CG, DT, LAYOUT, EPI, AR>(),                        \
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT, AR>::SMEM_BYTES,                                          \
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT, AR>::STAGES,                                              \
+     dg::GemmConfig<BN, CG, dg::sched_ints<KIND>(), DT, AR>::STAGE_BYTES}
+#define DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, EPI) DG_ENTRY_TLEA(BN, KIND, CG, DT, LAYOUT, EPI, dg::BM)
+#define DG_SMALL_A(BN) DG_ENTRY_TLEA(BN, dg::kDense, 1, dg::kE4M3, 0, 0, 64)
 #define DG_ENTRY_TL(BN, KIND, CG, DT, LAYOUT) DG_ENTRY_TLE(BN, KIND, CG, DT, LAYOUT, 0)
 #define DG_ENTRY_T(BN, KIND, CG, DT) DG_ENTRY_TL(BN, KIND, CG, DT, 0)
 #define DG_ACC(BN, CG) DG_ENTRY_TLE(BN, dg::kDense, CG, dg::kE4M3, 0, 1)
@@ -145,6 +149,8 @@ const KernelEntry kKernels[] = {
     DG_LAYOUT(128, 1), DG_LAYOUT(256, 1), DG_LAYOUT(128, 2), DG_LAYOUT(256, 2), DG_LAYOUT(128, 3), DG_LAYOUT(256, 3),
     DG_ACC(64, 1), DG_ACC(96, 1), DG_ACC(128, 1), DG_ACC(160, 1), DG_ACC(192, 1), DG_ACC(224, 1), DG_ACC(256, 1),
     DG_ACC(128, 2), DG_ACC(160, 2), DG_ACC(192, 2), DG_ACC(224, 2), DG_ACC(240, 2), DG_ACC(256, 2),
+    DG_SMALL_A(64), DG_SMALL_A(96), DG_SMALL_A(128), DG_SMALL_A(160), DG_SMALL_A(192), DG_SMALL_A(224),
+    DG_SMALL_A(256),
 };
 constexpr int kNumKernels = sizeof(kKernels) / sizeof(kKernels[0]);
 // 240 (a 16-column tail chunk, double-buffered at nearly 256 columns) is built
@@ -214,6 +220,10 @@ dg_status setup_device(int dev, DeviceState& st) {
                 }
                 st.max_clusters[i][s] = clusters;
             }
+            if (g_log && e.epi == 0)
+                std::fprintf(stderr, "[dgb200] BN=%d A-rows=%d: co-resident clusters of 2..8 CTAs: %d %d %d %d %d %d %d\n",
+                             e.bn, e.a_rows, st.max_clusters[i][2], st.max_clusters[i][3], st.max_clusters[i][4],
+                             st.max_clusters[i][5], st.max_clusters[i][6], st.max_clusters[i][7], st.max_clusters[i][8]);
         }
     }
     void* status = nullptr;
@@ -322,8 +332,12 @@ constexpr double kL2BytesPerClk = 77.0;
 // Tensor-core clocks lost per tile when the accumulator is single-buffered
 // (the MMA warp waits for the epilogue's TMEM reads).
 constexpr double kSingleBufferBubble = 600.0;
-// Fewest clocks per block-scaled MMA issued from the MMA warp (small N).
+// Fewest clocks per block-scaled MMA issued from the MMA warp (small N). A
+// single CTA streaming a small-M problem (64-row A stages) measured ~150: on
+// 64x7168x16384 with 64-wide tiles, 112 CTAs moved 2.97 TB/s, i.e. 8 KB of B
+// per ~600 clocks of four MMAs.
 constexpr double kMinMmaClocks = 98.0;
+constexpr double kMinMmaClocksSmallA = 150.0;
 // HBM bytes per SM clock for the whole GPU (~6.5 TB/s at ~1.85 GHz).
 constexpr double kHbmBytesPerClk = 3500.0;
 // When each B tile is read once (a single m-tile: small M), the weights stream
@@ -350,8 +364,8 @@ constexpr double kDsmemBytesPerClk = 32.0;
 // each, but no less than ~98 clocks per MMA issued; a pair's MMA covers 128
 // rows on each of its two SMs) and the L2 feed of the stage (rows_a rows of A
 // and bn/cg rows of B, 128 bytes each).
-double kblock_clocks(int bn, int cg, int rows_a) {
-    const double per_mma = bn / 2.0 > kMinMmaClocks ? bn / 2.0 : kMinMmaClocks;
+double kblock_clocks(int bn, int cg, int rows_a, double min_mma = kMinMmaClocks) {
+    const double per_mma = bn / 2.0 > min_mma ? bn / 2.0 : min_mma;
     const double tc = 4.0 * per_mma;
     const double l2 = (rows_a + static_cast<double>(bn) / cg) * 128.0 / kL2BytesPerClk;
     return tc > l2 ? tc : l2;
@@ -400,6 +414,11 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
     for (int i = 0; i < kNumKernels; ++i) {
         const KernelEntry& e = kKernels[i];
         if (e.kind != kind || e.dt != dt || e.layout != layout || e.epi != epi) continue;
+        // 64-row A stages serve exactly the dense NT calls with M <= 64 (unless
+        // CTA pairs are forced), which use no other kernels
+        const bool small_a_call =
+            kind == dg::kDense && layout == 0 && epi == 0 && dt == dg::kE4M3 && rows <= 64 && forced_cg != 2;
+        if ((e.a_rows < dg::BM) != small_a_call) continue;
         if (forced_bn != 0 && e.bn != forced_bn) continue;
         if (forced_cg != 0 && e.cg != forced_cg) continue;
         if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
@@ -414,7 +433,7 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
         const long long nb = (n + e.bn - 1) / e.bn;
         const long long tiles = mt * nb;
         const int rows_a = rows < dg::BM ? rows : dg::BM;
-        const double kbc0 = kblock_clocks(e.bn, e.cg, rows_a);
+        const double kbc0 = kblock_clocks(e.bn, e.cg, rows_a, e.a_rows < dg::BM ? kMinMmaClocksSmallA : kMinMmaClocks);
         const double bubble = num_acc_for(e.bn) == 1 ? kSingleBufferBubble : 0.0;
         const bool cluster_mode = scratch.mode == dg::SPLIT_CLUSTER;
         const int max_splits = cluster_mode ? kMaxClusterSplits : kMaxSplits;
@@ -549,7 +568,8 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     if (p.k_rotate) p.sf_vec4 = 0;                     // quads are walked in K order
     if (e->layout & 1) {
         if (!encode_mnmajor(&p.tma_a, a, a_rows, static_cast<uint64_t>(p.k))) return DG_ERR_INVALID_ARG;
-    } else if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats, 128, e->dt)) {
+    } else if (!encode_kmajor(&p.tma_a, a, a_rank, static_cast<uint64_t>(p.k), a_rows, a_mats,
+                              static_cast<uint32_t>(e->a_rows), e->dt)) {
         return DG_ERR_INVALID_ARG;
     }
     if (e->layout & 2) {
@@ -594,9 +614,9 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     if (g_log)
         std::fprintf(stderr,
                      "[dgb200] form=%d rows=%d N=%d K=%d groups=%d: BN=%d CTA-group=%d splits=%d (mode %d) grid=%d "
-                     "(units %d) smem=%d\n",
+                     "(units %d) smem=%d stages=%d A-rows=%d\n",
                      kind, p.rows, p.n, p.k, p.groups, bn, cg, choice.splits, p.split_mode, units * cg, choice.units,
-                     e->smem);
+                     e->smem, e->stages, e->a_rows);
     cudaError_t err = cudaLaunchKernelExC(&cfg, e->fn, args);
     return err == cudaSuccess ? DG_OK : DG_ERR_CUDA;
 }

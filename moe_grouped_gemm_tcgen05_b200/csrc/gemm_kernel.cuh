@@ -142,13 +142,18 @@ __host__ __device__ constexpr int sched_ints() {
                                              : (KIND == kContiguous ? MAX_CACHED_BLOCKS + 8 : 16);
 }
 
-template <int BN, int CG, int SCHED_INTS, int DT = kE4M3>
+// A_ROWS: rows of A per stage. 128 normally; 64 for the dense form when M <= 64
+// (a 64-row TMA box; the MMA still reads 128 rows, and its other 64 rows read
+// the next 8 KB of shared memory, whose accumulator rows are never stored).
+// The smaller stage keeps more weight bytes in flight per SM.
+template <int BN, int CG, int SCHED_INTS, int DT = kE4M3, int A_ROWS = BM>
 struct GemmConfig {
+    static_assert(A_ROWS == BM || A_ROWS == 64, "A stages of 128 or 64 rows");
     static_assert(BN % 16 == 0 && BN >= 32 && BN <= 256, "N tile must be a multiple of 16 in [32, 256]");
     static_assert(BN % 32 == 0 || CG == 2, "tiles with a 16-column tail chunk are built for CTA pairs");
     static_assert(CG == 1 || CG == 2, "one CTA or a CTA pair");
     static constexpr int B_ROWS = BN / CG;                      // rows of B in this CTA's shared memory
-    static constexpr int A_BYTES = BM * BK;
+    static constexpr int A_BYTES = A_ROWS * BK;
     static constexpr int B_BYTES = B_ROWS * BK;
     static constexpr int SFB_CHUNKS = (BN + 127) / 128;         // 128-column chunks of B scales (full width)
     static constexpr int SFA_BYTES = 512;                       // 32 rows x 16 bytes
@@ -162,7 +167,8 @@ struct GemmConfig {
     static constexpr int FIXED_BYTES =
         1024 /*align slack*/ + EPI_BYTES + SF_RING * SF_SLOT_BYTES + 512 /*barriers*/ + SCHED_BYTES;
     static constexpr int STAGES_FIT = (SMEM_LIMIT - FIXED_BYTES) / STAGE_BYTES;
-    static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+    static constexpr int MAX_STAGES = A_ROWS < BM ? 16 : 8;
+    static constexpr int STAGES = STAGES_FIT > MAX_STAGES ? MAX_STAGES : STAGES_FIT;
     static_assert(STAGES >= 2, "pipeline too shallow");
     static constexpr int SMEM_BYTES = FIXED_BYTES + STAGES * STAGE_BYTES;
 
@@ -659,7 +665,8 @@ __device__ __forceinline__ bool cluster_split_epilogue(const GemmParams& p, cons
 // atoms of M or N by K rows and described to the MMA as such.
 // EPI 1: the epilogue of D = C + A.B^T (optional C, bf16 or fp32 D; dense form);
 // EPI 0: plain bf16 D.
-template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0>
+// AR: rows of A per stage (64: dense, M <= 64, NT, plain epilogue; see GemmConfig).
+template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0, int AR = BM>
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
     static_assert(CG == 1 || (KIND != kMasked && KIND != kPsum), "CTA pairs are built for the dense and contiguous forms");
     static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
@@ -668,7 +675,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     static_assert(EPI == 0 || (KIND == kDense && DT == kE4M3 && LAYOUT == 0), "C / fp32 epilogue: dense NT form");
     constexpr bool kMnA = (LAYOUT & 1) != 0;
     constexpr bool kMnB = (LAYOUT & 2) != 0;
-    using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT>;
+    static_assert(AR == BM || (KIND == kDense && CG == 1 && DT == kE4M3 && LAYOUT == 0 && EPI == 0),
+                  "64-row A stages: dense NT form, single CTAs, plain epilogue");
+    using Cfg = GemmConfig<BN, CG, sched_ints<KIND>(), DT, AR>;
     // instruction descriptor with the operands' major modes
     constexpr uint32_t kIdesc = Cfg::IDESC | (kMnA ? (1u << 15) : 0u) | (kMnB ? (1u << 16) : 0u);
     // MN-major descriptor strides: one atom is 128 K-rows x 128 bytes of M or
@@ -683,7 +692,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* smem_a = smem;                                         // STAGES x 16 KB
+    uint8_t* smem_a = smem;                                         // STAGES x 16 KB (8 KB for 64-row A)
     uint8_t* smem_b = smem_a + STAGES * Cfg::A_BYTES;               // STAGES x B_ROWS*128
     uint8_t* smem_epi = smem_b + STAGES * Cfg::B_BYTES;             // 4 warps x 2 x 2 KB (1024-aligned)
     uint8_t* smem_sf = smem_epi + Cfg::EPI_BYTES;                   // SF_RING x (A scales, B scales)

@@ -55,7 +55,8 @@ def ref_dense(p):
 
 
 @pytest.mark.parametrize("bn", BLOCK_NS)
-@pytest.mark.parametrize("mnk", [(128, 256, 512), (300, 400, 1024), (257, 264, 640)])
+@pytest.mark.parametrize("mnk", [(128, 256, 512), (300, 400, 1024), (257, 264, 640),
+                                 (64, 264, 1024), (17, 400, 640)])   # M <= 64: 64-row A stages
 def test_dense_parity_every_tile_width(bn, mnk):
     p = W.dense(*mnk, seed=sum(mnk))
     d = run_dense(p, bn)
