@@ -195,8 +195,8 @@ DG_API dg_status fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, c
  * An operand stored M- or N-contiguous is loaded in 128-byte swizzle atoms of
  * that dimension and fed to the MMA as an MN-major operand (no transposition
  * pass). Limits as fp8_gemm_nt, plus M % 16 == 0 when A is stored [K, M] and
- * N % 16 == 0 when B is stored [K, N] (16-byte row pitch). Single CTAs, no
- * split-K; N tile 128 or 256.
+ * N % 16 == 0 when B is stored [K, N] (16-byte row pitch). No split-K; N tile
+ * 128 or 256 on single CTAs, 256 on CTA pairs (dgb200_set_cta_group).
  */
 DG_API dg_status fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
                              int N, int K, void* stream);

@@ -132,6 +132,7 @@ struct KernelEntry {
 #define DG_ENTRY_T(BN, KIND, CG, DT) DG_ENTRY_TL(BN, KIND, CG, DT, 0)
 #define DG_ACC(BN, CG) DG_ENTRY_TLE(BN, dg::kDense, CG, dg::kE4M3, 0, 1)
 #define DG_LAYOUT(BN, LAYOUT) DG_ENTRY_TL(BN, dg::kDense, 1, dg::kE4M3, LAYOUT)
+#define DG_LAYOUT_PAIR(BN, LAYOUT) DG_ENTRY_TL(BN, dg::kDense, 2, dg::kE4M3, LAYOUT)
 #define DG_ENTRY(BN, KIND, CG) DG_ENTRY_T(BN, KIND, CG, dg::kE4M3)
 #define DG_BF16_MASKED(BN) DG_ENTRY_T(BN, dg::kMasked, 1, dg::kBF16)
 #define DG_ALL_KINDS(BN) \
@@ -147,6 +148,7 @@ const KernelEntry kKernels[] = {
     DG_BF16_MASKED(64), DG_BF16_MASKED(96), DG_BF16_MASKED(128), DG_BF16_MASKED(160),
     DG_BF16_MASKED(192), DG_BF16_MASKED(224), DG_BF16_MASKED(256),
     DG_LAYOUT(128, 1), DG_LAYOUT(256, 1), DG_LAYOUT(128, 2), DG_LAYOUT(256, 2), DG_LAYOUT(128, 3), DG_LAYOUT(256, 3),
+    DG_LAYOUT_PAIR(256, 1), DG_LAYOUT_PAIR(256, 2), DG_LAYOUT_PAIR(256, 3),
     DG_ACC(64, 1), DG_ACC(96, 1), DG_ACC(128, 1), DG_ACC(160, 1), DG_ACC(192, 1), DG_ACC(224, 1), DG_ACC(256, 1),
     DG_ACC(128, 2), DG_ACC(160, 2), DG_ACC(192, 2), DG_ACC(224, 2), DG_ACC(240, 2), DG_ACC(256, 2),
     DG_SMALL_A(64), DG_SMALL_A(96), DG_SMALL_A(128), DG_SMALL_A(160), DG_SMALL_A(192), DG_SMALL_A(224),

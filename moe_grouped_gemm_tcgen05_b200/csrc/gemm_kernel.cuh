@@ -670,8 +670,8 @@ template <int BN, int KIND, int CG, int DT, int LAYOUT = 0, int EPI = 0, int AR 
 __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(const __grid_constant__ GemmParams p) {
     static_assert(CG == 1 || (KIND != kMasked && KIND != kPsum), "CTA pairs are built for the dense and contiguous forms");
     static_assert(DT == kE4M3 || (KIND == kMasked && CG == 1), "BF16 operands are built for the masked form");
-    static_assert(LAYOUT == 0 || (KIND == kDense && CG == 1 && DT == kE4M3), "layouts: dense, single CTAs");
-    static_assert(!(LAYOUT & 2) || BN % 128 == 0, "an MN-major B tile is whole 128-byte atoms");
+    static_assert(LAYOUT == 0 || (KIND == kDense && DT == kE4M3), "layouts: dense form");
+    static_assert(!(LAYOUT & 2) || (BN / CG) % 128 == 0, "an MN-major B tile is whole 128-byte atoms per CTA");
     static_assert(EPI == 0 || (KIND == kDense && DT == kE4M3 && LAYOUT == 0), "C / fp32 epilogue: dense NT form");
     constexpr bool kMnA = (LAYOUT & 1) != 0;
     constexpr bool kMnB = (LAYOUT & 2) != 0;
@@ -919,11 +919,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                         }
                     } else {
                         // the leader arms its barrier for both CTAs' bytes; both
-                        // CTAs' loads complete on the leader's barrier
+                        // CTAs' loads complete on the leader's barrier. An
+                        // MN-major operand is one 128-byte atom per CTA: {M or
+                        // N, K} box coordinates.
                         if (leader) mbar_arrive_expect_tx(&full_bar[stage], Cfg::TX_BYTES);
                         const uint32_t fb = full_leader0 + 8u * static_cast<uint32_t>(stage);
-                        tma_load_2d_pair(a_dst, &p.tma_a, fb, kx, a_row);
-                        if constexpr (KIND == kDense) {
+                        if constexpr (kMnA) tma_load_2d_pair(a_dst, &p.tma_a, fb, a_row, kx);
+                        else tma_load_2d_pair(a_dst, &p.tma_a, fb, kx, a_row);
+                        if constexpr (kMnB) {
+                            tma_load_2d_pair(b_dst, &p.tma_b, fb, b_row, kx);
+                        } else if constexpr (KIND == kDense) {
                             tma_load_2d_pair(b_dst, &p.tma_b, fb, kx, b_row);
                         } else {
                             tma_load_3d_pair(b_dst, &p.tma_b, fb, kx, b_row, g);

@@ -126,15 +126,17 @@ def test_accumulate_epilogue_stays_inside_d(mnk, bn, cg, splits, out_f32):
     check_fp(out.d.to(torch.float64).cpu().numpy(), c_host + _ref_dense(p), f"acc {mnk}")
 
 
+@pytest.mark.parametrize("cg", [1, 2])
 @pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
-def test_operand_layouts_stay_inside_d(layout):
+def test_operand_layouts_stay_inside_d(layout, cg):
     M, N, K = 208, 400, 1024
     p = W.dense(M, N, K, seed=9)
+    dg.set_cta_group(cg)
     a = p["a"] if layout[0] == "n" else np.ascontiguousarray(p["a"].T)
     b = p["b"] if layout[1] == "t" else np.ascontiguousarray(p["b"].T)
     out = Guarded(M, N)
     getattr(dg, f"fp8_gemm_{layout}")(_dev(a), _pack_dev(p["sfa_f32"]), _dev(b), _pack_dev(p["sfb_f32"]), out.d)
-    out.check_bands(f"layout {layout}")
+    out.check_bands(f"layout {layout} cg={cg}")
     check_fp(bf16_to_f64(out.d), _ref_dense(p), f"layout {layout}")
 
 

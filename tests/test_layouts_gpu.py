@@ -24,6 +24,7 @@ def _reset():
     dg.device_error(clear=True)
     yield
     dg.set_block_n(0)
+    dg.set_cta_group(0)
     dg.set_splits(0)
     assert dg.device_error(clear=True) == 0
 
@@ -33,9 +34,9 @@ def _dev(x):
 
 
 @pytest.mark.parametrize("layout", ["nn", "tn", "tt"])
-@pytest.mark.parametrize("bn", [128, 256])
-@pytest.mark.parametrize("mnk", [(128, 256, 512), (272, 400, 1024), (512, 768, 2048)])
-def test_layout_parity_and_equal_to_nt(layout, bn, mnk):
+@pytest.mark.parametrize("bn,cg", [(128, 1), (256, 1), (256, 2)])
+@pytest.mark.parametrize("mnk", [(128, 256, 512), (272, 400, 1024), (512, 768, 2048), (400, 528, 640)])
+def test_layout_parity_and_equal_to_nt(layout, bn, cg, mnk):
     M, N, K = mnk
     p = W.dense(M, N, K, seed=M + 5 * N + K + bn)
     a_mk, b_nk = p["a"], p["b"]
@@ -44,6 +45,7 @@ def test_layout_parity_and_equal_to_nt(layout, bn, mnk):
     sfa = dg.pack_ue8m0(_dev(p["sfa_f32"]))
     sfb = dg.pack_ue8m0(_dev(p["sfb_f32"]))
     dg.set_block_n(bn)
+    dg.set_cta_group(cg)   # 2: CTA pairs, a 256-row tile with one 128-byte atom of A and of B per CTA
     d = fill_sentinel(torch.empty((M, N), dtype=torch.bfloat16, device="cuda"))
     FN[layout](_dev(a), sfa, _dev(b), sfb, d)
     d_nt = torch.empty_like(d)
@@ -52,7 +54,7 @@ def test_layout_parity_and_equal_to_nt(layout, bn, mnk):
     torch.cuda.synchronize()
     assert not is_sentinel(d).any()
     ref = oracle.fp8_gemm(a, oracle.pack_ue8m0(p["sfa_f32"]), b, oracle.pack_ue8m0(p["sfb_f32"]), layout)
-    check_fp(bf16_to_f64(d), ref, f"{layout} {mnk} bn={bn}")
+    check_fp(bf16_to_f64(d), ref, f"{layout} {mnk} bn={bn} cg={cg}")
     assert torch.equal(d.view(torch.int16), d_nt.view(torch.int16)), f"{layout} differs from nt"
 
 
