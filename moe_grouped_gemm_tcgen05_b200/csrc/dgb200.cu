@@ -348,6 +348,10 @@ constexpr double kHbmBytesPerClk = 3500.0;
 // issue to arrival; all CTAs together draw about 2400 bytes per clock.
 constexpr double kHbmLatencyClk = 4400.0;
 constexpr double kBStreamBytesPerClk = 2400.0;
+// One SM streams weights at no more than ~24 bytes per clock (~45 GB/s):
+// M = 64 problems measured 40-48 GB/s per streaming SM, so a choice that
+// leaves SMs idle cannot make up for them with a faster stream per SM.
+constexpr double kBStreamPerSmBytesPerClk = 24.0;
 // Split-K through global scratch (fp8_gemm_nt_noalloc): the most ranges per
 // tile; the unit that reduces a tile pays about one L2 round trip (~700
 // clocks) per 32 columns per two splits, plus a fixed hand-off (fence,
@@ -467,8 +471,10 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
                 const double active = static_cast<double>(work < su ? work : su);
                 const double lat = kHbmLatencyClk / e.stages;
                 const double bw = static_cast<double>(e.bn / e.cg) * 128.0 * active / kBStreamBytesPerClk;
+                const double per_sm = static_cast<double>(e.bn / e.cg) * 128.0 / kBStreamPerSmBytesPerClk;
                 if (lat > kbc) kbc = lat;
                 if (bw > kbc) kbc = bw;
+                if (per_sm > kbc) kbc = per_sm;
             }
             double unit = kb_unit * kbc + bubble;
             if (splits > 1) {
