@@ -564,6 +564,8 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     // would read each weight tile from DRAM only once, thrash L2 with A and
     // read more, 592 MB against 473 MB)
     p.raster_group = 16 / cg;
+    p.raster_shift = cg == 2 ? 3 : 4;
+    p.inv_band_tiles = 1.0f / static_cast<float>(p.raster_group * p.num_n_blocks);
     p.wait_limit_ns = g_wait_limit_ns.load();
     p.test_mode = g_test_mode.load();
     p.splits = choice.splits;

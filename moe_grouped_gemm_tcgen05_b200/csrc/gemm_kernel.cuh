@@ -109,7 +109,9 @@ struct GemmParams {
     int sfb_per_row;          // 1: one scale row per row of B (1x128 blocks); 0: per 128x128 block
     int num_m_blocks;         // ceil(rows / (128 * CG)) m-tiles
     int num_n_blocks;         // ceil(N / BN)
-    int raster_group;         // m-tiles per raster band (dense / contiguous)
+    int raster_group;         // m-tiles per raster band (dense / contiguous), a power of two
+    int raster_shift;         // log2(raster_group)
+    float inv_band_tiles;     // 1 / (raster_group * num_n_blocks), for the band index
     uint64_t wait_limit_ns;   // bound of every mbarrier wait
     int k_rotate;             // 1: each tile walks its K groups starting at group (tile mod groups)
     int test_mode;            // 1: CTA 0 withholds its first scale-group arrive (exercises the timeout path)
@@ -255,23 +257,46 @@ __device__ __forceinline__ void sleep_ns(uint64_t ns) {
 // Dense / contiguous: banded raster. Within a band of `raster_group` m-tiles
 // the m-tile varies fastest, so CTAs running at the same time share the B tile
 // and a bounded slab of A.
+// The arithmetic is kept free of integer divisions where it can be (each
+// costs ~0.1 us of a lone warp's time, paid between two tiles): no split
+// needs none, the band index comes from a float reciprocal corrected to the
+// exact quotient (below 2^20 tiles, where one correction step suffices), and
+// full bands (a power-of-two number of m-tiles) use a shift.
 __device__ __forceinline__ bool raster_tile(const GemmParams& p, int t_unit, Tile& c) {
-    const int t = t_unit / p.splits;          // output tile; its splits are consecutive work units
-    const int split = t_unit - t * p.splits;
+    const int kgc = (p.kb + 3) / 4;  // K groups of four 128-K blocks
+    int t = t_unit;                  // output tile; its splits are consecutive work units
+    int split = 0;
+    c.kg0 = 0;
+    c.kg1 = kgc;
+    if (p.splits > 1) {
+        t = t_unit / p.splits;
+        split = t_unit - t * p.splits;
+        c.kg0 = split * kgc / p.splits;
+        c.kg1 = (split + 1) * kgc / p.splits;
+    }
     const int total = p.num_m_blocks * p.num_n_blocks;
     if (t >= total) return false;
     c.base = t;
     c.split = split;
-    const int kgc = (p.kb + 3) / 4;  // K groups of four 128-K blocks
-    c.kg0 = split * kgc / p.splits;
-    c.kg1 = (split + 1) * kgc / p.splits;
     const int band_tiles = p.raster_group * p.num_n_blocks;
-    const int band = t / band_tiles;
+    int band;
+    if (total < (1 << 20)) {
+        band = __float2int_rz(__int2float_rn(t) * p.inv_band_tiles);
+        if ((band + 1) * band_tiles <= t) ++band;
+        if (band * band_tiles > t) --band;
+    } else {
+        band = t / band_tiles;
+    }
     const int local = t - band * band_tiles;
     const int m0 = band * p.raster_group;
     const int gm = min(p.raster_group, p.num_m_blocks - m0);
-    c.n_blk = local / gm;
-    c.m_blk = m0 + (local - c.n_blk * gm);
+    if (gm == p.raster_group) {
+        c.n_blk = local >> p.raster_shift;
+        c.m_blk = m0 + (local & (gm - 1));
+    } else {
+        c.n_blk = local / gm;
+        c.m_blk = m0 + (local - c.n_blk * gm);
+    }
     c.g = 0;
     return true;
 }
