@@ -54,10 +54,12 @@ SHAPES = [(64, 512, 4096),     # 8 groups, one m-block
           (130, 1024, 3200)]   # 7 groups (last one partial: 25 K-blocks), M tail
 
 
-@pytest.mark.parametrize("splits", [2, 3, 5, 8])
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("splits", [2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("bn", [64, 96, 128, 256])
 @pytest.mark.parametrize("mnk", SHAPES)
 def test_split_k_parity(mnk, bn, splits):
+    # every cluster size (2..8 CTAs) at several tile widths: pieces of 8
+    # columns dealt unevenly among the CTAs, 64-row A stages for M <= 64
     M, N, K = mnk
     groups = (K // 128 + 3) // 4
     if splits > groups:
