@@ -21,7 +21,9 @@ Also reported:
                FP8/BF16 dense ratio), from MEASURED_PEAKS.json
   e2e          the same metric through the Python binding with pinned HOST
                buffers: every step copies A, B and fp32 scales host->device,
-               packs both scale tensors, runs the GEMM and copies D back
+               packs both scale tensors, runs the GEMM and copies D back, with
+               copies and compute of different problems overlapped on three
+               streams
   cpu_baseline the CPU oracle (numpy float64) on a bounded sample: the first
                rows of A against all of B for each problem
   clocks       NVML SM clock and throttle reasons sampled during the timed region
@@ -280,7 +282,13 @@ def steady_state_us(torch, dg, p, max_copies=32, replays=5):
 
 
 def run_e2e(torch, dg, probs, steps):
-    """Same metric through the binding with pinned host buffers and copies in the timed region."""
+    """Same metric through the binding with pinned host buffers and copies in
+    the timed region. Every step copies each problem's A, B and fp32 scales in,
+    packs both scale tensors, runs the GEMM and copies D out. The three kinds
+    of work run on three streams ordered by events, so that the copies of one
+    problem overlap the compute of another (PCIe is full duplex): copy-in of
+    problem i waits until the previous step's GEMM i has consumed its inputs,
+    and GEMM i waits until the previous step's D_i has been copied out."""
     host = []
     for p in probs:
         h = {k: p[k].cpu().pin_memory() for k in ("a", "sfa_f32", "b", "sfb_f32")}
@@ -291,23 +299,44 @@ def run_e2e(torch, dg, probs, steps):
         dev.append({k: torch.empty_like(p[k]) for k in ("a", "sfa_f32", "b", "sfb_f32", "sfa", "sfb", "d")})
     h2d = sum(sum(h[k].numel() * h[k].element_size() for k in ("a", "sfa_f32", "b", "sfb_f32")) for h in host)
     d2h = sum(h["d"].numel() * h["d"].element_size() for h in host)
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(probs)
+    ev_in = [torch.cuda.Event() for _ in range(n)]     # inputs of problem i on the device
+    ev_cmp = [torch.cuda.Event() for _ in range(n)]    # GEMM i done (inputs consumed, D written)
+    ev_out = [torch.cuda.Event() for _ in range(n)]    # D_i copied out
+    for i in range(n):
+        ev_cmp[i].record(s_cmp)
+        ev_out[i].record(s_out)
 
     def one_step():
-        for h, d in zip(host, dev):
-            for k in ("a", "sfa_f32", "b", "sfb_f32"):
-                d[k].copy_(h[k], non_blocking=True)
-            dg.pack_ue8m0(d["sfa_f32"], d["sfa"])
-            dg.pack_ue8m0(d["sfb_f32"], d["sfb"])
-            dg.fp8_gemm_nt(d["a"], d["sfa"], d["b"], d["sfb"], d["d"])
-            h["d"].copy_(d["d"], non_blocking=True)
+        for i, (h, d) in enumerate(zip(host, dev)):
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(ev_cmp[i])
+                for k in ("a", "sfa_f32", "b", "sfb_f32"):
+                    d[k].copy_(h[k], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[i])
+                s_cmp.wait_event(ev_out[i])
+                dg.pack_ue8m0(d["sfa_f32"], d["sfa"])
+                dg.pack_ue8m0(d["sfb_f32"], d["sfb"])
+                dg.fp8_gemm_nt(d["a"], d["sfa"], d["b"], d["sfb"], d["d"])
+                ev_cmp[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[i])
+                h["d"].copy_(d["d"], non_blocking=True)
+                ev_out[i].record(s_out)
 
     one_step()
     torch.cuda.synchronize()
+    # the timed region: from before the first copy-in to after the last copy-out
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
+    s.record(s_in)
     for _ in range(steps):
         one_step()
-    e.record()
+    s_in.wait_event(ev_out[n - 1])
+    s_in.wait_event(ev_cmp[n - 1])
+    e.record(s_in)
     torch.cuda.synchronize()
     ms = s.elapsed_time(e) / steps
     return ms, h2d, d2h
