@@ -863,13 +863,19 @@ def committed_traffic(key):
 
 
 def dg_kernel_rev():
-    """Hash of the kernel sources; a committed ncu traffic figure counts only for this revision."""
+    """Hash of the kernel sources with their comments and blank lines removed;
+    a committed ncu traffic figure counts only for this revision."""
     import hashlib
+    import re
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "moe_grouped_gemm_tcgen05_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        code = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(name.encode() + b"\0" + code.encode())
     return h.hexdigest()[:12]
 
 

@@ -38,7 +38,8 @@
  * time, since no compute call except fp8_gemm_nt_noalloc touches memory other
  * than its own arguments and the status word.
  *
- * CUDA Graph capture. Every compute entry point is capture safe: no host
+ * CUDA Graph capture. Every compute entry point of the method (all but
+ * fp8_gemm_nt_noalloc, about which no claim is made) is capture safe: no host
  * synchronisation, no allocation, no host reads of device values, and a launch
  * configuration fixed by the scalar sizes alone ("DeepGEMM CUDA Graph
  * Compatibility for Masked Grouped GEMMs: Implementation Guide", sections
@@ -252,8 +253,7 @@ DG_API dg_status fp8_gemm_nt_acc(const void* a, const int32_t* sfa, const void* 
  * running when the next one starts on another stream) race on it and give
  * wrong results. Calls on one stream are ordered and safe.
  * The first call on a device does per-device set-up (kernel attributes,
- * symbol addresses; no allocation) and should come before any stream capture
- * that includes this call.
+ * symbol addresses; no allocation).
  */
 DG_API dg_status fp8_gemm_nt_noalloc(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
                                      int M, int N, int K, int splits, void* stream);

@@ -9,7 +9,8 @@ missing or cannot run on the current device, calls raise.
 Tensors are torch tensors used as device memory; work is queued on torch's
 current CUDA stream. No call synchronises or allocates (except the
 convenience allocations of ``pack_ue8m0`` / ``empty_*`` when no output is
-given), so the calls can be captured in a CUDA Graph.
+given), so the calls of the method can be captured in a CUDA Graph (no claim
+is made for ``fp8_gemm_nt_noalloc``).
 """
 
 from __future__ import annotations

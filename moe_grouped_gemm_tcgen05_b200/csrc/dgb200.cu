@@ -4,7 +4,8 @@
 // the TMA tensor maps (driver entry point, no libcuda link), picks a tile
 // width from the sizes and the SM count, and launches one kernel on the
 // caller's stream. A compute call allocates nothing, never synchronises and
-// reads no device value, so it can be captured in a CUDA Graph. The library
+// reads no device value, so the calls of the method can be captured in a CUDA
+// Graph (no claim is made for fp8_gemm_nt_noalloc). The library
 // allocates no device memory at all: split-K adds its partial tiles inside a
 // thread-block cluster (distributed shared memory), and the device status word
 // and the scratch of fp8_gemm_nt_noalloc are static __device__ variables.
