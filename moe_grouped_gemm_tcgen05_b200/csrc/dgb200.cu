@@ -314,6 +314,19 @@ bool encode_mnmajor(CUtensorMap* map, const void* base, uint64_t mn, uint64_t k)
     return r == CUDA_SUCCESS;
 }
 
+// fp32 output of the dense form (and its C), in boxes of 32 columns x 16 rows
+// (128 bytes per row) with the 128-byte swizzle.
+bool encode_d_f32(CUtensorMap* map, const void* base, uint64_t n, uint64_t rows) {
+    cuuint64_t dims[2] = {n, rows};
+    cuuint64_t strides[1] = {4 * n};
+    cuuint32_t box[2] = {32, 16};
+    cuuint32_t elem[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // bf16 output, written by TMA in 32x32 boxes with the 64-byte swizzle.
 bool encode_d_bf16(CUtensorMap* map, void* base, int rank, uint64_t n, uint64_t rows, uint64_t mats) {
     cuuint64_t dims[3] = {n, rows, mats};
@@ -590,6 +603,15 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
         return DG_ERR_INVALID_ARG;
     }
     if (!encode_d_bf16(&p.tma_d, p.d, a_rank, static_cast<uint64_t>(p.n), a_rows, a_mats)) return DG_ERR_INVALID_ARG;
+    if (kind == dg::kDense && p.out_f32 &&
+        !encode_d_f32(&p.tma_d, p.d32, static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.rows)))
+        return DG_ERR_INVALID_ARG;
+    if (kind == dg::kDense && p.c != nullptr) {
+        const bool ok = p.out_f32 ? encode_d_f32(&p.tma_c, p.c, static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.rows))
+                                  : encode_d_bf16(&p.tma_c, const_cast<void*>(p.c), 2, static_cast<uint64_t>(p.n),
+                                                  static_cast<uint64_t>(p.rows), 1);
+        if (!ok) return DG_ERR_INVALID_ARG;
+    }
     // contiguous pairs walk two passes (see next_tile in gemm_kernel.cuh)
     const long long tiles = (cg == 1 ? max_tiles_per_nblock : p.num_m_blocks) * static_cast<long long>(p.num_n_blocks) *
                             choice.splits * (cg == 2 && kind == dg::kContiguous ? 2 : 1);

@@ -95,7 +95,9 @@ constexpr int MAX_CLUSTER_SPLITS = 8;   // portable cluster size
 struct GemmParams {
     CUtensorMap tma_a;        // A: 2-D {K, rows} (dense, contiguous, psum_m) or 3-D {K, max_m, G} (masked)
     CUtensorMap tma_b;        // B: 2-D {K, N} (dense) or 3-D {K, N, G} (grouped); box BN/CG rows
-    CUtensorMap tma_d;        // D (bf16, store): 2-D {N, rows} or 3-D {N, max_m, G}; 32x32 box, 64-byte swizzle
+    CUtensorMap tma_d;        // D (store): 2-D {N, rows} or 3-D {N, max_m, G}; bf16: 32x32 boxes, 64-byte
+                              //   swizzle; fp32 (dense): 32 columns x 16 rows, 128-byte swizzle
+    CUtensorMap tma_c;        // C of D = C + A.B^T (load), D's type and box; set when c is given
     const int32_t* sfa;       // packed scale rows of A
     const int32_t* sfb;       // packed scale rows of B (per 128 rows or per row, per group)
     __nv_bfloat16* d;         // output
@@ -732,7 +734,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
     uint64_t* epi_bar = drain_bar + 1;               // split-K: the four epilogue warps meet
     uint64_t* red_free = epi_bar + 1;                // cluster split-K: every peer's ring is free
     uint64_t* red_full = red_free + 1;               // cluster split-K: peers' pieces landed, per epilogue warp
-    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(red_full + 4);
+    uint64_t* cbar = red_full + 4;                   // D = C + A.B^T: a C piece landed, per epilogue warp
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(cbar + 4);
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_tmem + 1);
     volatile int* s_last = reinterpret_cast<volatile int*>(s_tmem + 2);  // split-K: this unit reduces
     int* s_prefix = reinterpret_cast<int*>(s_tmem + 4);             // [groups + 1] (masked, psum_m)
@@ -761,6 +764,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         }
         mbar_init(drain_bar, 1);
         mbar_init(epi_bar, 4);
+        if constexpr (EPI == 1)
+            for (int q = 0; q < 4; ++q) mbar_init(&cbar[q], 1);
         if constexpr (KIND == kDense && CG == 1) {
             if (p.split_mode == SPLIT_CLUSTER) {
                 // one arrive from each peer; per epilogue warp, one arrive (made
@@ -782,6 +787,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         tma_prefetch_desc(&p.tma_a);
         tma_prefetch_desc(&p.tma_b);
         tma_prefetch_desc(&p.tma_d);
+        if (EPI == 1 && p.c != nullptr) tma_prefetch_desc(&p.tma_c);
     }
     if (warp == 1) {
         tmem_alloc<CG>(s_tmem, Cfg::TMEM_COLS);
@@ -1200,6 +1206,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         // the MMA warp right after the last read, and then writes bf16:
         // 32x32 chunks staged in swizzled shared memory and stored with TMA
         // when all 32 rows may be written, predicated 16-byte stores otherwise.
+        // D = C + A.B^T (dense) moves C in and D out through the same staging
+        // buffers with TMA (row-wise 16-byte loads and stores of 32 rows at a
+        // time measured 10-19% slower on 4096x7168x16384: their many small
+        // requests slow the operand loads of the tile being computed).
         const int q = static_cast<int>(warp & 3);   // TMEM sub-partition of this warp
         uint8_t* stg = smem_epi + (warp - 2) * Cfg::EPI_WARP_BYTES;
         [[maybe_unused]] uint32_t tempty_leader0 = 0;  // the leader's accumulator barriers (pairs)
@@ -1209,6 +1219,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
         uint32_t epi_phase = 0;
         int gcur = 0;
         int buf = 0;
+        [[maybe_unused]] uint32_t c_phase = 0;   // D = C + A.B^T: parity of this warp's C barrier
+        bool e_abort = false;                     // a wait inside a chunk's output gave up
         Tile c;
         for (int t = unit; next_tile<KIND, true, CG>(p, s_prefix, s_mm, t, units, gcur, c, lane); t += units) {
             const int row_coord = c.m_blk * BM * CG + my_rows + 32 * q;
@@ -1313,85 +1325,137 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
             // column hc, written as one 32x32 chunk
             auto emit32 = [&](const uint32_t* v, int hc) {
                 const int col = n0 + hc;
-                if (col >= p.n) return;  // warp-uniform: N tail
+                if (col >= p.n || e_abort) return;  // warp-uniform: N tail
                 float f[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
                 if constexpr (EPI == 1) {
-                    if (p.c != nullptr && valid) {
-                        // + C (N % 8 == 0: whole 8-column pieces are in or out)
-                        const size_t at = out_row * static_cast<size_t>(p.n) + col;
-                        if (p.out_f32) {
-                            const float* crow = static_cast<const float*>(p.c) + at;
-#pragma unroll
-                            for (int q8 = 0; q8 < 4; ++q8) {
-                                if (col + 8 * q8 >= p.n) continue;
-                                const float4 x0 = *reinterpret_cast<const float4*>(crow + 8 * q8);
-                                const float4 x1 = *reinterpret_cast<const float4*>(crow + 8 * q8 + 4);
-                                f[8 * q8] += x0.x; f[8 * q8 + 1] += x0.y; f[8 * q8 + 2] += x0.z; f[8 * q8 + 3] += x0.w;
-                                f[8 * q8 + 4] += x1.x; f[8 * q8 + 5] += x1.y; f[8 * q8 + 6] += x1.z; f[8 * q8 + 7] += x1.w;
+                    // dense form: C comes in and D goes out through the warp's two
+                    // 2 KB staging buffers with TMA
+                    if (p.out_f32) {
+                        // 32 fp32 columns as two boxes of 16 rows x 128 bytes (the
+                        // 128-byte swizzle: granule g of row r at g ^ (r & 7)), rows
+                        // 0-15 in the first buffer and 16-31 in the second
+                        if (lane == 0) bulk_wait_group_read<0>();  // both buffers free
+                        __syncwarp();
+                        uint8_t* sb = stg + (lane >> 4) * 2048 + (lane & 15) * 128;
+                        const uint32_t sw8 = lane & 7u;
+                        if (p.c != nullptr) {
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(&cbar[q], 4096);
+                                tma_load_2d(stg, &p.tma_c, &cbar[q], col, row_coord);
+                                tma_load_2d(stg + 2048, &p.tma_c, &cbar[q], col, row_coord + 16);
                             }
-                        } else {
-                            const __nv_bfloat16* crow = static_cast<const __nv_bfloat16*>(p.c) + at;
+                            if (!wait_warp(&cbar[q], c_phase, p, s_abort)) {
+                                e_abort = true;
+                                return;
+                            }
+                            c_phase ^= 1u;
 #pragma unroll
-                            for (int q8 = 0; q8 < 4; ++q8) {
-                                if (col + 8 * q8 >= p.n) continue;
-                                const uint4 x = *reinterpret_cast<const uint4*>(crow + 8 * q8);
+                            for (int g = 0; g < 8; ++g) {
+                                const float4 x = *reinterpret_cast<const float4*>(sb + 16 * (g ^ sw8));
+                                f[4 * g] += x.x;
+                                f[4 * g + 1] += x.y;
+                                f[4 * g + 2] += x.z;
+                                f[4 * g + 3] += x.w;
+                            }
+                        }
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            *reinterpret_cast<float4*>(sb + 16 * (g ^ sw8)) =
+                                make_float4(f[4 * g], f[4 * g + 1], f[4 * g + 2], f[4 * g + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tma_d, stg, col, row_coord);
+                            tma_store_2d(&p.tma_d, stg + 2048, col, row_coord + 16);
+                            bulk_commit_group();
+                        }
+                    } else {
+                        // bf16: one 32-row x 64-byte box (64-byte swizzle, as below)
+                        // per chunk, buffers taken in turn
+                        const uint32_t sw = (lane >> 1) & 3u;
+                        // the store issued two chunks ago has finished reading this buffer
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        uint8_t* sb = stg + buf * 2048;
+                        if (p.c != nullptr) {
+                            if (lane == 0) {
+                                mbar_arrive_expect_tx(&cbar[q], 2048);
+                                tma_load_2d(sb, &p.tma_c, &cbar[q], col, row_coord);
+                            }
+                            if (!wait_warp(&cbar[q], c_phase, p, s_abort)) {
+                                e_abort = true;
+                                return;
+                            }
+                            c_phase ^= 1u;
+#pragma unroll
+                            for (int g = 0; g < 4; ++g) {
+                                const uint4 x = *reinterpret_cast<const uint4*>(sb + lane * 64 + 16 * (g ^ sw));
                                 const uint32_t w4[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
                                 for (int h2 = 0; h2 < 4; ++h2) {
-                                    const float2 c2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
-                                    f[8 * q8 + 2 * h2] += c2.x;
-                                    f[8 * q8 + 2 * h2 + 1] += c2.y;
+                                    const float2 c2 =
+                                        __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[h2]));
+                                    f[8 * g + 2 * h2] += c2.x;
+                                    f[8 * g + 2 * h2 + 1] += c2.y;
                                 }
                             }
                         }
-                    }
-                    if (p.out_f32) {
-                        if (valid) {
-                            float* drow32 = p.d32 + out_row * static_cast<size_t>(p.n) + col;
 #pragma unroll
-                            for (int q4 = 0; q4 < 8; ++q4)
-                                if (col + 4 * q4 < p.n)
-                                    *reinterpret_cast<float4*>(drow32 + 4 * q4) =
-                                        make_float4(f[4 * q4], f[4 * q4 + 1], f[4 * q4 + 2], f[4 * q4 + 3]);
+                        for (int g = 0; g < 4; ++g) {
+                            uint32_t w4[4];
+#pragma unroll
+                            for (int h2 = 0; h2 < 4; ++h2) {
+                                __nv_bfloat162 b2 = __floats2bfloat162_rn(f[8 * g + 2 * h2], f[8 * g + 2 * h2 + 1]);
+                                w4[h2] = *reinterpret_cast<uint32_t*>(&b2);
+                            }
+                            *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
+                                make_uint4(w4[0], w4[1], w4[2], w4[3]);
                         }
-                        return;
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tma_d, sb, col, row_coord);
+                            bulk_commit_group();
+                        }
+                        buf ^= 1;
                     }
-                }
-                uint32_t w[16];
+                } else {
+                    uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-                    w[i] = *reinterpret_cast<uint32_t*>(&b2);
-                }
-                if (use_tma) {
-                    // the store issued two chunks ago has finished reading this buffer
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
-                    uint8_t* sb = stg + buf * 2048;
-                    // 32 rows x 64 bytes with the 64-byte swizzle: granule g of
-                    // row r sits at granule g ^ ((r >> 1) & 3)
-                    const uint32_t sw = (lane >> 1) & 3u;
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
-                            make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
-                        else if constexpr (KIND == kPsum) tma_store_2d(&p.tma_d, sb, col, s_mm[c.g] + row_coord);
-                        else tma_store_2d(&p.tma_d, sb, col, row_coord);
-                        bulk_commit_group();
+                    for (int i = 0; i < 16; ++i) {
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+                        w[i] = *reinterpret_cast<uint32_t*>(&b2);
                     }
-                    buf ^= 1;
-                } else if (valid) {
+                    if (use_tma) {
+                        // the store issued two chunks ago has finished reading this buffer
+                        if (lane == 0) bulk_wait_group_read<1>();
+                        __syncwarp();
+                        uint8_t* sb = stg + buf * 2048;
+                        // 32 rows x 64 bytes with the 64-byte swizzle: granule g of
+                        // row r sits at granule g ^ ((r >> 1) & 3)
+                        const uint32_t sw = (lane >> 1) & 3u;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        if (col + 8 * q4 < p.n)
-                            *reinterpret_cast<uint4*>(drow + hc + 8 * q4) =
-                                make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                        for (int g = 0; g < 4; ++g)
+                            *reinterpret_cast<uint4*>(sb + lane * 64 + 16 * (g ^ sw)) =
+                                make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (KIND == kMasked) tma_store_3d(&p.tma_d, sb, col, row_coord, c.g);
+                            else if constexpr (KIND == kPsum) tma_store_2d(&p.tma_d, sb, col, s_mm[c.g] + row_coord);
+                            else tma_store_2d(&p.tma_d, sb, col, row_coord);
+                            bulk_commit_group();
+                        }
+                        buf ^= 1;
+                    } else if (valid) {
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            if (col + 8 * q4 < p.n)
+                                *reinterpret_cast<uint4*>(drow + hc + 8 * q4) =
+                                    make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                    }
                 }
             };
             // the 16-column tail chunk of a 240-wide tile (pairs, dense form):
@@ -1519,8 +1583,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                     }
                 }
             }
+            if (e_abort) break;
             if (++acc == NUM_ACC) { acc = 0; acc_phase ^= 1u; }
         }
+        // a C load whose wait gave up may still land: let it, within a bound,
+        // before shared memory goes away
+        if (e_abort) wait_quiet(&cbar[q], c_phase, p.wait_limit_ns / 16);
         // every bulk store must have completed before the CTA exits
         if (lane == 0) bulk_wait_group<0>();
         __syncwarp();

@@ -2,6 +2,8 @@
 for profilers (e.g. ncu) and quick timing.
 
     python -m moe_grouped_gemm_tcgen05_b200.profile_case dense --m 4096 --n 7168 --k 16384 --iters 3 [--cta-group 2]
+    python -m moe_grouped_gemm_tcgen05_b200.profile_case dense ... --acc-f32     # D = C + A.B^T, fp32, in place
+    python -m moe_grouped_gemm_tcgen05_b200.profile_case dense ... --sfb-per-row # one weight scale row per row of B
     python -m moe_grouped_gemm_tcgen05_b200.profile_case masked --groups 32 --max-m 256 --expected-m 96 --n 4096 --k 7168
     python -m moe_grouped_gemm_tcgen05_b200.profile_case contiguous --groups 8 --n 4096 --k 7168
 
@@ -33,6 +35,8 @@ def main(argv=None):
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--block-n", type=int, default=0)
     ap.add_argument("--cta-group", type=int, default=0, help="dense only: 1 = single CTAs, 2 = CTA pairs")
+    ap.add_argument("--acc-f32", action="store_true", help="dense only: D = C + A.B^T in fp32, accumulated in place")
+    ap.add_argument("--sfb-per-row", action="store_true", help="dense only: B scaled per row (1x128 blocks)")
     args = ap.parse_args(argv)
 
     torch.cuda.set_device(0)
@@ -44,6 +48,12 @@ def main(argv=None):
         sfa, sfb = dg.pack_ue8m0(p["sfa_f32"]), dg.pack_ue8m0(p["sfb_f32"])
         d = torch.empty((args.m, args.n), dtype=torch.bfloat16, device="cuda")
         call = lambda: dg.fp8_gemm_nt(p["a"], sfa, p["b"], sfb, d)
+        if args.acc_f32:
+            d32 = torch.zeros((args.m, args.n), dtype=torch.float32, device="cuda")
+            call = lambda: dg.fp8_gemm_nt_acc(p["a"], sfa, p["b"], sfb, d32, c=d32)
+        elif args.sfb_per_row:
+            sfb_rows = sfb.repeat_interleave(128, dim=0)[: args.n].contiguous()
+            call = lambda: dg.fp8_gemm_nt_sfb_gran(p["a"], sfa, p["b"], sfb_rows, d, 1)
     elif args.form == "masked":
         mm = W.masked_m_uniform(W.rng_for(1003), G=args.groups, expected=args.expected_m)
         mm = np.minimum(mm, args.max_m)
