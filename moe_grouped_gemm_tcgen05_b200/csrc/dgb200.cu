@@ -90,12 +90,15 @@ const int g_k_rotate = [] {
     const char* v = std::getenv("DGB200_K_ROTATE");
     return (v != nullptr && v[0] == '1') ? 1 : 0;
 }();
-// With B scaled per row, scale rows whose length is a multiple of 4 words, on
-// 16-byte aligned bases, are read 16 bytes (four K groups) per row at a time
-// when the K groups are walked in order; DGB200_SF_VEC4=0 reads one word per
-// group instead. Measured on 4096x7168x16384 (BN 224, CTA pairs): per-row B
-// scales 370 -> 335 us; with 128x128 B blocks (one broadcast word per 128
-// columns) the one-word reads are faster, 311 vs 325 us, so they keep them.
+// Scale rows whose length is a multiple of 4 words, on 16-byte aligned bases,
+// are read 16 bytes (four K groups) per row at a time when the K groups are
+// walked in order: A's rows always (dense form), B's rows when B is scaled per
+// row (every form); with 128x128 B blocks, B's broadcast words are read per
+// group. DGB200_SF_VEC4=0 reads one word per row and group instead. Measured
+// on 4096x7168x16384 (BN 224, CTA pairs; the leader reads the scale rows of
+// 256 rows of A, which do not stay in L1 between groups): 316 -> 308 us with
+// 128x128 B blocks, 384 -> 359 us with per-row B scales. (Reading B's
+// broadcast words 16 bytes at a time too measured slower, 325 vs 311 us.)
 const bool g_sf_vec4 = [] {
     const char* v = std::getenv("DGB200_SF_VEC4");
     return !(v != nullptr && v[0] == '0');
@@ -568,8 +571,8 @@ dg_status launch_gemm_with(const TileChoice& choice, float* ws, uint32_t* counte
     p.kp = (p.kb + 3) / 4;
     p.nb_sf = p.sfb_per_row ? p.n : (p.n + 127) / 128;
     // 16-byte reads of the scale rows need every row to start on a 16-byte boundary
-    p.sf_vec4 = (p.sfb_per_row && e->dt == dg::kE4M3 && g_sf_vec4 && p.kp % 4 == 0 && aligned(p.sfa, 16) &&
-                 aligned(p.sfb, 16))
+    p.sf_vec4 = ((p.sfb_per_row || kind == dg::kDense) && e->dt == dg::kE4M3 && g_sf_vec4 && p.kp % 4 == 0 &&
+                 aligned(p.sfa, 16) && (!p.sfb_per_row || aligned(p.sfb, 16)))
                     ? 1
                     : 0;
     p.num_n_blocks = (p.n + bn - 1) / bn;

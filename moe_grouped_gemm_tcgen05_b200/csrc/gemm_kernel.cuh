@@ -435,6 +435,11 @@ struct ScaleWords {
                 ap[j] = static_cast<uint32_t>(__ldg(p.sfa + (row_base + rp) * p.kp + kg));
             }
         }
+        load_b(p, n0, g, kg, lane);
+    }
+
+    // B's words of group kg only
+    __device__ __forceinline__ void load_b(const GemmParams& p, int n0, int g, int kg, uint32_t lane) {
         const int32_t* sfb = p.sfb + static_cast<size_t>(KIND == kDense ? 0 : max(g, 0)) * p.nb_sf * p.kp;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
@@ -470,8 +475,10 @@ struct ScaleWords {
 // for packed rows whose length is a multiple of four words on 16-byte
 // aligned bases. Same rows and columns as ScaleWords; `base` is the first of
 // the four groups (a multiple of 4). One such load serves four groups, so the
-// scattered row reads are a quarter of the one-word loads: this pays when B
-// is scaled per row, where every column reads its own scale row.
+// scattered row reads are a quarter of the one-word loads: this pays for A's
+// rows, and for B's when B is scaled per row (every column reads its own
+// scale row). With 128x128 B blocks the B words, one broadcast word per 128
+// columns, are read per group (`b_words`).
 template <int BN, int KIND, int CG>
 struct ScaleQuads {
     static constexpr int CH = (BN + 127) / 128;
@@ -479,6 +486,7 @@ struct ScaleQuads {
     uint4 ap[CG == 2 ? 4 : 1];
     uint4 b[CH][4];
     int lo, hi;  // the groups [lo, hi) of the tile that this quad serves
+    int n0, g;   // the tile's first column and group
 
     __device__ __forceinline__ static const uint4* at(const int32_t* row_start, int base) {
         return reinterpret_cast<const uint4*>(row_start + base);
@@ -496,6 +504,9 @@ struct ScaleQuads {
                 ap[j] = __ldg(at(p.sfa + (row_base + rp) * p.kp, base));
             }
         }
+        this->n0 = n0;
+        this->g = g;
+        if (!p.sfb_per_row) return;  // B words are read per group
         const int32_t* sfb = p.sfb + static_cast<size_t>(KIND == kDense ? 0 : max(g, 0)) * p.nb_sf * p.kp;
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch) {
@@ -512,12 +523,17 @@ struct ScaleQuads {
         return static_cast<uint32_t>(i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w)));
     }
 
-    // the words of group base + i
-    __device__ __forceinline__ void words(ScaleWords<BN, KIND, CG>& w, int i) const {
+    // the words of group base + i (kg)
+    __device__ __forceinline__ void words(const GemmParams& p, ScaleWords<BN, KIND, CG>& w, int i, int kg,
+                                          uint32_t lane) const {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             w.a[j] = pick(a[j], i);
             if constexpr (CG == 2) w.ap[j] = pick(ap[j], i);
+        }
+        if (!p.sfb_per_row) {
+            w.load_b(p, n0, g, kg, lane);
+            return;
         }
 #pragma unroll
         for (int ch = 0; ch < CH; ++ch)
@@ -1058,7 +1074,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) fp8_block_scaled_gemm_kernel(c
                 auto put_quad = [&](const ScaleQuads<BN, KIND, CG>& q) -> bool {
                     for (int kg = q.lo; kg < q.hi; ++kg) {
                         ScaleWords<BN, KIND, CG> w;
-                        q.words(w, kg & 3);
+                        q.words(p, w, kg & 3, kg, lane);
                         if (!put(w)) return false;
                     }
                     return true;
