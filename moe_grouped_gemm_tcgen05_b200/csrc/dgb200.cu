@@ -442,6 +442,15 @@ TileChoice choose_tile_in(const DeviceState* st, int kind, int rows, int n, int 
         const bool small_a_call =
             kind == dg::kDense && layout == 0 && epi == 0 && dt == dg::kE4M3 && rows <= 64 && forced_cg != 2;
         if ((e.a_rows < dg::BM) != small_a_call) continue;
+        // M <= 64 calls all take 128-column tiles (the split count is still
+        // chosen per shape): a small GEMM's first operand loads land several
+        // microseconds later when the previous GEMM ran another kernel
+        // (cold instruction fetch), which outweighs what a shape-specific
+        // width gains alone. Measured on the dense step of 8 problems (four
+        // with M = 64): 700 against 730 us per step (median of 21 replays,
+        // the one-width step faster in 16 of 21 pairs), although
+        // 64x24576x1536 alone takes 13.2 instead of 11.2 us.
+        if (small_a_call && forced_bn == 0 && e.bn != 128) continue;
         if (forced_bn != 0 && e.bn != forced_bn) continue;
         if (forced_cg != 0 && e.cg != forced_cg) continue;
         if (forced_cg == 0 && e.cg == 2 && rows < 256) continue;  // a pair needs two row blocks
