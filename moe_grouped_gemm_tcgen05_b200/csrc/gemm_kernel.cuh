@@ -478,7 +478,7 @@ struct ScaleWords {
 // scattered row reads are a quarter of the one-word loads: this pays for A's
 // rows, and for B's when B is scaled per row (every column reads its own
 // scale row). With 128x128 B blocks the B words, one broadcast word per 128
-// columns, are read per group (`b_words`).
+// columns, are read per group (`words` calls ScaleWords::load_b).
 template <int BN, int KIND, int CG>
 struct ScaleQuads {
     static constexpr int CH = (BN + 127) / 128;
